@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Decode-attention throughput: history tokens/s and achieved HBM GB/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload exact|hybrid|ragged|tiny]
+                    [--variant auto|simt|mma] [--impl ours|reference]
+
+A step is one decode step of the whole hot path over one batch: split attention over
+every tier (exact BF16 and, for hybrid workloads, the compact tier) followed by the exact
+log-sum-exp merge.  The default workload is the exact-tier GQA decode: batch 8, 32 query
+/ 8 KV heads, d 128, 8192 BF16 tokens per sequence, 512-token splits (268 MB of K/V per
+step, larger than the 126 MB L2, so no flush is needed between steps).
+
+One process per GPU (torchrun for N > 1): every rank runs an independent replica on its
+own batch (the batch partitions with no exchange), so scaling is weak and the reported
+value is the tokens of all ranks over the slowest rank's time.  Rank 0 prints one JSON
+line.  ``--impl reference`` times the float64 CPU oracle on this host's cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention history tokens/s/GPU & achieved HBM GB/s vs B200 peak"
+UNIT = "history tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "simt", "mma"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--soak-seconds", type=float, default=1.5,
+                    help="untimed steady-state run before the timed region (clocks settle, samples taken)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------------
+# clocks sampled during the run
+# ----------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, name):
+        self.marks.append((name, time.monotonic()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for t, line in self.lines:
+            if t0 <= t <= t1:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.lower() == "active"})
+        pw = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------------
+
+
+def make_workload(name: str, device, rank: int):
+    from kv_cache_tiering_b200 import synth, workloads
+    base = synth.WORKLOADS[name]
+    wl = synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.d, base.split_tokens, seed=base.seed + rank,
+                        extra=dict(base.extra))
+    if name in ("exact", "tiny"):
+        w = workloads.ExactResident(wl, device)
+        tokens = w.B * w.T
+    elif name == "hybrid":
+        w = workloads.HybridResident(wl, device)
+        tokens = w.B * w.T
+    else:
+        w = workloads.RaggedPaged(wl, device)
+        tokens = int(w.lens.sum())
+    return wl, w, tokens
+
+
+def describe(name, wl, w):
+    d = {"workload": {
+        "exact": "exact-tier GQA decode: batch 8, 32 q / 8 KV heads, d 128, 8192 BF16 tokens, contiguous, 512-token splits",
+        "tiny": "tiny exact decode: batch 1, 1 q / 1 KV head, d 64, 256 BF16 tokens, 4 splits of 64",
+        "hybrid": "hybrid tier: batch 4, 32 q / 8 KV heads, d 128, 32768 tokens (newest 2048 BF16, 30720 4-bit codes)",
+        "ragged": "ragged paged hybrid: batch 64, lengths U[1024, 65536], 16-token pages, newest 1024 BF16",
+    }[name], "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.d, "split_tokens": wl.split_tokens,
+        "kv_bytes_per_step": w.kv_bytes()}
+    d["l2"] = ("inputs larger than the 126 MB L2, no flush" if w.kv_bytes() > 126e6
+               else "L2 flushed (256 MB write) before every step")
+    return d
+
+
+# ----------------------------------------------------------------------------------
+# reference arm: the float64 CPU oracle
+# ----------------------------------------------------------------------------------
+
+
+def oracle_sequence_fn(name, wl, seed_rank=0):
+    """Return (fn(i) -> tokens processed, n_units, description) running the oracle on unit i."""
+    import numpy as np
+    from kv_cache_tiering_b200 import synth
+    from oracle import akv_oracle as ora
+    f64 = ora.bf16_bits_to_f64
+    if name in ("exact", "tiny"):
+        T = wl.extra["T"]
+        q = synth.queries(wl)
+
+        def fn(i):
+            b = i % wl.B
+            k, v = synth.history_head_major(wl, b, T)
+            ora.decode_sequence(f64(q[b]), [(f64(k), f64(v))], wl.scale, wl.split_tokens)
+            return T
+        return fn, wl.B, "one sequence (all heads, all splits, merge) per unit"
+    if name == "hybrid":
+        T, W = wl.extra["T"], wl.extra["window"]
+        q = synth.queries(wl)
+
+        def fn(i):
+            b = i % wl.B
+            k, v = synth.history_head_major(wl, b, T)
+            h = i % wl.Hkv
+            G = wl.Hq // wl.Hkv
+            ek, ev = ora.encode(k[h, :T - W]), ora.encode(v[h, :T - W])
+            kh, vh = ora.dequantize(ek.codes, ek.scale_bits)[None], ora.dequantize(ev.codes, ev.scale_bits)[None]
+            tiers = [(kh, vh), (f64(k[h:h + 1, T - W:]), f64(v[h:h + 1, T - W:]))]
+            ora.decode_sequence(f64(q[b, h * G:(h + 1) * G]), tiers, wl.scale, wl.split_tokens)
+            return T / wl.Hkv
+        return fn, wl.B * wl.Hkv, "one (sequence, KV head) with its 4 query heads per unit, encode included"
+    lens = synth.ragged_lengths(wl)
+    q = synth.queries(wl)
+
+    def fn(i):
+        b = int(np.argsort(lens)[i * (wl.B - 1) // 7]) if i < 8 else i % wl.B
+        L = int(lens[b])
+        Wn = min(L, wl.extra["window"])
+        k, v = synth.history_head_major(wl, b, L, key_dist="student_t")
+        h = 0
+        ek, ev = ora.encode(k[h, :L - Wn]), ora.encode(v[h, :L - Wn])
+        kh, vh = ora.dequantize(ek.codes, ek.scale_bits)[None], ora.dequantize(ev.codes, ev.scale_bits)[None]
+        tiers = [(kh, vh), (f64(k[h:h + 1, L - Wn:]), f64(v[h:h + 1, L - Wn:]))]
+        ora.decode_sequence(f64(q[b, :4]), tiers, wl.scale, wl.split_tokens)
+        return L / wl.Hkv
+    return fn, 8, "one KV head of one sequence per unit, 8 sequences spread over the length range"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(name, wl, budget_s: float = 15.0, max_units=None):
+    fn, n_units, desc = oracle_sequence_fn(name, wl)
+    tokens, units = 0.0, 0
+    t0 = time.perf_counter()
+    while units < (max_units or n_units):
+        tokens += fn(units)
+        units += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return tokens / dt, units, desc, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from kv_cache_tiering_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    fn, n_units, desc = oracle_sequence_fn(args.workload, wl)
+    for i in range(args.warmup):
+        fn(i)
+    times, tokens = [], 0.0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        tokens += fn(i)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = tokens / total
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "reference": "float64 numpy oracle on the host CPU",
+                       "step": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} units: {desc}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------
+
+
+def run_ours(args):
+    import torch
+    from kv_cache_tiering_b200 import akv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    variant = {"auto": akv.AKV_VARIANT_AUTO, "simt": akv.AKV_VARIANT_SIMT, "mma": akv.AKV_VARIANT_MMA}[args.variant]
+    wl, w, tokens = make_workload(args.workload, dev, rank)
+    step = w.step
+    stream = torch.cuda.current_stream()
+    flush = None
+    if w.kv_bytes() <= 126e6:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def one_step():
+        if flush is not None:
+            flush.fill_(1)
+        step.step(w.q, variant, stream)
+
+    launches_per_step = sum(1 for t in step.tiers if int(sum(t.lens)) > 0) + 1  # attends + merge (B <= 256)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(3, args.warmup)):
+        one_step()
+    torch.cuda.synchronize()
+    # soak: steady-state steps before the timed region
+    t_soak = time.monotonic()
+    while time.monotonic() - t_soak < args.soak_seconds:
+        for _ in range(20):
+            one_step()
+        torch.cuda.synchronize()
+
+    n_ev = args.steps
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.monotonic()
+    start.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        a0[i].record(stream)
+        step.attend(w.q, variant, stream)
+        a1[i].record(stream)
+        step.merge(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.monotonic()
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    attend_ms = [a0[i].elapsed_time(a1[i]) for i in range(args.steps)]
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    # post-timed soak so the sampler has points inside the loaded window
+    t_post = time.monotonic()
+    while time.monotonic() - t_post < 0.3:
+        for _ in range(20):
+            one_step()
+        torch.cuda.synchronize()
+    err = int(step.err.item())
+
+    # ---- end to end through the public API: pinned host q in, O and LSE out, every step
+    q_host = torch.from_numpy(w.q_bits.view("int16")).pin_memory()
+    o_host = torch.empty(step.o.shape, dtype=torch.float32).pin_memory()
+    lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(w.q)
+    for _ in range(3):
+        q_dev.copy_(q_host, non_blocking=True)
+        one_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        q_dev.copy_(q_host, non_blocking=True)
+        if flush is not None:
+            flush.fill_(1)
+        step.step(q_dev, variant, stream)
+        o_host.copy_(step.o, non_blocking=True)
+        lse_host.copy_(step.lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    sampler.stop()
+
+    total_tokens = tokens * world * args.steps
+    value = total_tokens / (ms * 1e-3)
+    e2e_value = total_tokens / (e2e_ms * 1e-3)
+    peak, peak_kind = peaks()
+    attend_avg_ms = sum(attend_ms) / len(attend_ms)
+    kv_bytes = w.kv_bytes()
+    achieved = kv_bytes / (attend_avg_ms * 1e-3) / 1e9
+    clocks = sampler.summary(t_soak, t_wall1 + 0.3)
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": dict(describe(args.workload, wl, w), parallelism=f"independent replicas x{world}",
+                               accumulate="f32", variant=args.variant),
+                "hbm_gbs": kv_bytes * world * args.steps / (ms * 1e-3) / 1e9,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "kernel": "akv attend (all tiers of a step)",
+                             "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+                             "attend_ms_avg": attend_avg_ms},
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(q_host.numel() * 2),
+                        "d2h_bytes_per_step": int(o_host.numel() * 4 + lse_host.numel() * 4)},
+                "gpu_launches": launches_per_step * args.steps,
+                "clocks": clocks, "device_error_word": err}
+        if world == 1 and not args.no_cpu_baseline:
+            cv, units, desc, dt = time_oracle(args.workload, wl)
+            line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                    "sample": f"{units} units ({desc}), {dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

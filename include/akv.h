@@ -1,0 +1,242 @@
+/*
+ * akv.h -- C ABI of libakv: tiered KV-history decode attention for NVIDIA B200 (sm_100a).
+ *
+ * One decode step attends a single new query per head over a long key/value history.
+ * The history lives in tiers ("Context beyond VRAM", section "What I built": two
+ * precision tiers with separate contracts):
+ *   - an exact tier, BF16 keys and values, bit-identical to fully resident attention;
+ *   - a compact tier for older history: each (token, KV head) vector is rotated by a
+ *     Walsh-Hadamard transform, scaled by its L2 norm (stored as binary16) and coded as
+ *     4-bit indices into a fixed 16-level Lloyd-Max table for N(0,1).  The GPU reads the
+ *     codes directly; the query is rotated instead of the keys ("QuantForge V2
+ *     Walkthrough", section 1 "Triton Fused Kernels": rotation preserves dot products).
+ * Each tier is attended in fixed-size splits; every split writes a partial output and its
+ * log-sum-exp ("Bringing a serving stack up on new silicon", section "What I built": the
+ * attention statistic the memory layer needs), and the partials are merged exactly
+ * ("Context beyond VRAM", "What I built": merged with exact attention arithmetic).
+ * Older history can be staged from pinned host memory through a bounded device region
+ * whose buffers are released only after every copy and kernel that touched them has
+ * finished ("Context beyond VRAM", sections "My approach" and "What I built").
+ *
+ * Conventions for every call:
+ *   - The caller owns all device memory and pinned host memory.  The library allocates
+ *     no device memory; a stager owns only CUDA events and a small host struct.
+ *   - Device pointers are plain CUDA device addresses.  Host arrays (lens, slot bases)
+ *     are read during the call and not retained.
+ *   - Work is enqueued on the caller's stream; no call synchronises the device except
+ *     the stager's bounded waits and akv_stager_destroy.
+ *   - Arguments are validated before anything is launched.  A refused call launches
+ *     nothing and returns a negative akv_status; akv_last_error() (thread-local) then
+ *     holds a one-line reason.  Errors found on the device (a page id outside the pool, a
+ *     non-finite input) set bits of a caller-provided device int32 error word, which the
+ *     caller reads after the stream has reached that point; akv_error_word_status maps
+ *     the word to a status.
+ *   - Supported shapes: head dim d in {64, 128}; G = Hq / Hkv in {1, 2, 4, 8}; split_tokens
+ *     a multiple of 16 in [16, 1024].  Other shapes return AKV_ERR_UNSUPPORTED.
+ *   - Not thread-safe per object; independent calls from several threads are safe.
+ */
+#ifndef AKV_H_
+#define AKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define AKV_ABI_VERSION 1
+
+/* Opaque CUDA stream (cudaStream_t); 0 is the legacy default stream. */
+typedef struct CUstream_st* akv_stream_t;
+
+typedef enum akv_status {
+  AKV_OK = 0,
+  AKV_ERR_INVALID = -1,      /* malformed argument (null pointer, negative size, misaligned) */
+  AKV_ERR_UNSUPPORTED = -2,  /* valid but not implemented (head dim, group size, split size) */
+  AKV_ERR_CUDA = -3,         /* a CUDA runtime call failed; akv_last_error names it */
+  AKV_ERR_NOT_PINNED = -4,   /* a staging source is not page-locked host memory */
+  AKV_ERR_BUDGET = -5,       /* a chunk does not fit one staging buffer */
+  AKV_ERR_TIMEOUT = -6,      /* a staging buffer was still in use when the wait ran out */
+  AKV_ERR_NONFINITE = -7,    /* device: an encoded vector held inf or NaN */
+  AKV_ERR_RANGE = -8,        /* device: an encoded vector's norm overflows binary16 */
+  AKV_ERR_BOUNDS = -9        /* device: a page id outside [0, n_pages) */
+} akv_status;
+
+/* Bits of the device error word. */
+#define AKV_EFLAG_NONFINITE 0x1
+#define AKV_EFLAG_RANGE 0x2
+#define AKV_EFLAG_BOUNDS 0x4
+
+int akv_abi_version(void);
+const char* akv_last_error(void);
+const char* akv_status_string(int status);
+/* Most severe status encoded in an error word (AKV_OK for 0). */
+akv_status akv_error_word_status(int32_t word);
+
+/* The library's binary16 centroid table, ascending (host; 16 entries).  The library
+ * solves for the 16-level Lloyd-Max quantiser of N(0,1) on the host at load time, makes
+ * it odd-symmetric and rounds every level to binary16 (round to nearest even). */
+void akv_centroids_f16(uint16_t out[16]);
+
+/* ------------------------------------------------------------------------------------
+ * Tiers
+ * ------------------------------------------------------------------------------------ */
+
+enum { AKV_TIER_BF16 = 0, AKV_TIER_CODES4 = 1 };
+
+/* Tokens per page (paged tiers) and per code block (compact tier). */
+#define AKV_PAGE_TOKENS 16
+
+/* Bytes of one compact-tier block of 16 tokens for head dim d: 16 code rows of d/2 bytes
+ * (token order; byte k of a row holds code 2k in its low nibble and code 2k+1 in its
+ * high nibble), then 16 little-endian binary16 scales.  1056 bytes at d = 128. */
+#define AKV_CODES4_BLOCK_BYTES(d) (16 * ((d) / 2) + 32)
+
+/*
+ * One tier of the history of a batch of B sequences, for one layer.
+ *
+ * Addressing of token t (0-based within the tier) of sequence b, KV head h:
+ *   BF16, contiguous:   k + b*stride_seq + h*stride_head + t*stride_token        (elements)
+ *   BF16, paged:        k + P*stride_seq + h*stride_head + (t%16)*stride_token,
+ *                       P = page_table[b*page_table_stride + t/16]               (elements)
+ *   CODES4, contiguous: block k + b*stride_seq + h*stride_head + (t/16)*stride_token,
+ *                       row t%16 of that block                                   (blocks)
+ *   CODES4, paged:      block k + P*stride_seq + h*stride_head, row t%16         (blocks)
+ * The head dimension is contiguous.  V uses the same layout from base v.
+ * BF16 bases must be 16-byte aligned and BF16 strides multiples of 8 elements; CODES4
+ * bases must be 16-byte aligned.  Buffers must cover every addressed token: the library
+ * cannot see allocation sizes, except that paged tiers check page ids against n_pages.
+ *
+ * lens[b] (host) is the number of tokens of sequence b in this tier (0 allowed).
+ * slot_base[b] (host) is the partial-output slot of the tier's first split for sequence
+ * b; split s (tokens [s*split_tokens, (s+1)*split_tokens) of the tier) goes to slot
+ * slot_base[b] + s.  Splits are aligned to the start of the tier.
+ */
+typedef struct akv_tier {
+  int32_t kind;                  /* AKV_TIER_BF16 or AKV_TIER_CODES4 */
+  int32_t paged;                 /* 0 contiguous, 1 paged through page_table */
+  const void* k;                 /* device */
+  const void* v;                 /* device */
+  const int32_t* page_table;     /* device [B][page_table_stride], paged tiers only */
+  int64_t page_table_stride;     /* int32 entries between page-table rows */
+  int64_t n_pages;               /* pages in the pool (paged tiers) */
+  int64_t stride_seq;            /* contiguous: between sequences; paged: between pages */
+  int64_t stride_head;           /* between KV heads */
+  int64_t stride_token;          /* see the addressing above; ignored for paged CODES4 */
+  const int32_t* lens;           /* host [B] */
+  const int32_t* slot_base;      /* host [B] */
+} akv_tier;
+
+/* ------------------------------------------------------------------------------------
+ * akv_encode_history -- rotate, quantise and pack BF16 history into the compact tier.
+ *
+ * For every sequence b < B, KV head h < Hkv and token t < dst->lens[b], the BF16 key and
+ * value vectors x at token t of src are encoded into token t of dst (the compact form of
+ * the hybrid tier of "Context beyond VRAM", "What I built"):
+ *   z = H x (unnormalised Sylvester-order Walsh-Hadamard transform, float64 butterflies
+ *       h = 1, 2, ..., d/2 mapping (a, b) to (a + b, a - b));
+ *   s = binary16(sqrt(sum of x_i^2)), the sum taken in float64 by pairwise halving;
+ *   code_i = number of boundaries b_j = (c_j + c_{j+1}) / 2, j < 15, with z_i > s * b_j;
+ *   s == 0 gives codes 7.
+ * Every block touched is written whole: rows past dst->lens[b] in the last block hold the
+ * zero-vector encoding (codes 7, scale 0).  A vector with a non-finite coordinate or a
+ * norm that rounds to binary16 infinity is written as the zero-vector encoding and sets
+ * AKV_EFLAG_NONFINITE / AKV_EFLAG_RANGE in *err_word (device int32, may be NULL).
+ * src: kind BF16 (its lens and slot_base are not used).  dst: kind CODES4; its k and v
+ * blocks are WRITTEN.  Codes and scales are bit-exact against the float64 definition.
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, int Hkv, int d,
+                              int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * akv_decode_attend -- split-KV GQA decode attention over one or more tiers.
+ *
+ * q: device BF16 [B][Hq][d], contiguous.  Query head h reads KV head h / G, G = Hq/Hkv.
+ * For every tier, sequence b with lens[b] > 0, split s and query head h it writes
+ *   o_part[(slot*Hq + h)*d + i]  (float32)   and   lse_part[slot*Hq + h]  (float32)
+ * with slot = slot_base[b] + s:  scores_t = softmax_scale * q_h . k_t over the split's
+ * tokens, O = sum_t softmax(scores)_t v_t, LSE = ln sum_t exp(scores_t).  A compact tier
+ * is attended in the rotated basis (q rotated once per split, outputs rotated back), over
+ * the dequantised vectors x_hat = H (s * c[code] / sqrt d) / sqrt d.
+ * Every slot must lie in [0, n_slots); slots of different splits must not coincide.
+ * variant: AKV_VARIANT_AUTO (the faster path), AKV_VARIANT_SIMT (CUDA cores, float32
+ * FMA) or AKV_VARIANT_MMA (tensor-core mma.sync across the GQA group).  For a given
+ * variant and split layout the result does not depend on where the tokens are stored, so
+ * a staged run equals the resident run bit for bit.  Page ids outside [0, n_pages) set
+ * AKV_EFLAG_BOUNDS in *err_word (device, may be NULL) and read page 0 instead.
+ * ------------------------------------------------------------------------------------ */
+enum { AKV_VARIANT_AUTO = 0, AKV_VARIANT_SIMT = 1, AKV_VARIANT_MMA = 2 };
+
+akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
+                             const akv_tier* tiers, int n_tiers, int split_tokens,
+                             float* o_part, float* lse_part, int64_t n_slots, int variant,
+                             int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * akv_merge_lse -- exact log-sum-exp merge of split partials ("Context beyond VRAM",
+ * "What I built": the tiers are merged with exact attention arithmetic).
+ *
+ * For sequence b and head h the partials in slots seq_slot_base[b] .. +seq_n_slots[b]-1
+ * (host arrays) are merged in increasing slot order:
+ *   M = max_s LSE_s, w_s = exp(LSE_s - M), L = sum_s w_s,
+ *   o[(b*Hq + h)*d + i] = sum_s w_s O_s[i] / L,   lse[b*Hq + h] = M + ln L.
+ * No finite partial (seq_n_slots[b] == 0, or all -inf) gives O = 0 and LSE = -inf.
+ * o, lse: device float32 [B][Hq][d] and [B][Hq].
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_slots,
+                         const int32_t* seq_slot_base, const int32_t* seq_n_slots, int B, int Hq,
+                         int d, float* o, float* lse, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * akv_plan_slots -- host helper: the standard slot layout.
+ *
+ * Sequence-major: sequence b owns a contiguous run of slots holding tier 0's splits,
+ * then tier 1's, and so on (ceil(tier_lens[i][b] / split_tokens) splits per tier).
+ * Writes tier_slot_base[i][b], seq_slot_base[b], seq_n_slots[b] and *n_slots (all host).
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, int split_tokens,
+                          int32_t* const* tier_slot_base, int32_t* seq_slot_base,
+                          int32_t* seq_n_slots, int64_t* n_slots);
+
+/* ------------------------------------------------------------------------------------
+ * Staging: pinned host history through a bounded device region ("Context beyond VRAM",
+ * "My approach": pinned host memory is the authoritative copy and the GPU a bounded
+ * working set; "What I built": a buffer is released only after every copy and kernel
+ * that touched it has finished).
+ *
+ * The region (caller-owned device memory, 256-byte aligned) is cut into n_buffers equal
+ * buffers used round-robin.  Each buffer keeps the list of events recorded by the copies
+ * and consumers that touched it since it was last filled.
+ *
+ * akv_stage_chunk: take the next buffer; make sure every event on its list has fired;
+ *   copy `bytes` from pinned_src (page-locked host memory, else AKV_ERR_NOT_PINNED) with
+ *   cudaMemcpyAsync on copy_stream; record the copy's event.  bytes larger than one
+ *   buffer gives AKV_ERR_BUDGET.  timeout_ms >= 0: the host polls the events for at most
+ *   timeout_ms and returns AKV_ERR_TIMEOUT, leaving the buffer untouched, if one is still
+ *   pending.  timeout_ms < 0: the host does not wait; copy_stream waits for the events
+ *   on the device instead.  Returns the buffer index and its device address.
+ * akv_stager_use: make consumer_stream wait for the buffer's latest copy.
+ * akv_stager_release: record on consumer_stream that the consumer's work on the buffer
+ *   is enqueued; the buffer is reused only after that event fires.
+ * akv_stage_writeback: copy bytes from the buffer at byte offset to pinned host memory on
+ *   stream, ordered after the buffer's copy, and add the copy to the buffer's list.
+ * akv_stager_destroy: wait (host) for every listed event, then free the stager.
+ * All events are created with timing disabled (timing events serialise copies).
+ * ------------------------------------------------------------------------------------ */
+typedef struct akv_stager akv_stager;
+
+akv_status akv_stager_create(void* dev_region, size_t region_bytes, int n_buffers, akv_stager** out);
+akv_status akv_stage_chunk(akv_stager* st, const void* pinned_src, size_t bytes, akv_stream_t copy_stream,
+                           int timeout_ms, int* buf_index, void** dev_ptr);
+akv_status akv_stager_use(akv_stager* st, int buf_index, akv_stream_t consumer_stream);
+akv_status akv_stager_release(akv_stager* st, int buf_index, akv_stream_t consumer_stream);
+akv_status akv_stage_writeback(akv_stager* st, int buf_index, size_t offset, void* pinned_dst, size_t bytes,
+                               akv_stream_t stream);
+akv_status akv_stager_destroy(akv_stager* st);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AKV_H_ */

@@ -1,0 +1,268 @@
+"""ctypes binding of libakv (``include/akv.h``): argument marshalling only.
+
+Every computation runs in the CUDA library; this module converts torch tensors to
+device pointers, numpy/int sequences to host int32 arrays and torch streams to
+``cudaStream_t`` handles, and raises ``AkvError`` for a negative status.  There is no
+fallback: importing this module fails loudly when ``lib/libakv.so`` is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libakv.so")
+
+AKV_OK = 0
+AKV_ERR_INVALID = -1
+AKV_ERR_UNSUPPORTED = -2
+AKV_ERR_CUDA = -3
+AKV_ERR_NOT_PINNED = -4
+AKV_ERR_BUDGET = -5
+AKV_ERR_TIMEOUT = -6
+AKV_ERR_NONFINITE = -7
+AKV_ERR_RANGE = -8
+AKV_ERR_BOUNDS = -9
+
+AKV_EFLAG_NONFINITE = 0x1
+AKV_EFLAG_RANGE = 0x2
+AKV_EFLAG_BOUNDS = 0x4
+
+AKV_TIER_BF16 = 0
+AKV_TIER_CODES4 = 1
+AKV_VARIANT_AUTO = 0
+AKV_VARIANT_SIMT = 1
+AKV_VARIANT_MMA = 2
+PAGE_TOKENS = 16
+
+
+def codes4_block_bytes(d: int) -> int:
+    return 16 * (d // 2) + 32
+
+
+class AkvError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"akv status {status}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libakv.so not built ({_LIB_PATH}); run `python -m kv_cache_tiering_b200.build`")
+    return ctypes.CDLL(_LIB_PATH)
+
+
+lib = _load()
+
+_p = ctypes.c_void_p
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+
+class AkvTierC(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("paged", ctypes.c_int32),
+        ("k", _p),
+        ("v", _p),
+        ("page_table", _p),
+        ("page_table_stride", ctypes.c_int64),
+        ("n_pages", ctypes.c_int64),
+        ("stride_seq", ctypes.c_int64),
+        ("stride_head", ctypes.c_int64),
+        ("stride_token", ctypes.c_int64),
+        ("lens", _p),
+        ("slot_base", _p),
+    ]
+
+
+def _sig(name, res, *args):
+    f = getattr(lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_sig("akv_abi_version", ctypes.c_int)
+_sig("akv_last_error", ctypes.c_char_p)
+_sig("akv_status_string", ctypes.c_char_p, ctypes.c_int)
+_sig("akv_error_word_status", ctypes.c_int, ctypes.c_int32)
+_sig("akv_centroids_f16", None, ctypes.POINTER(ctypes.c_uint16))
+_sig("akv_plan_slots", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_p), ctypes.c_int,
+     ctypes.POINTER(_p), _p, _p, ctypes.POINTER(ctypes.c_int64))
+_sig("akv_encode_history", ctypes.c_int, ctypes.POINTER(AkvTierC), ctypes.POINTER(AkvTierC), ctypes.c_int,
+     ctypes.c_int, ctypes.c_int, _p, _p)
+_sig("akv_decode_attend", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, _p, ctypes.c_int64, ctypes.c_int, _p, _p)
+_sig("akv_merge_lse", ctypes.c_int, _p, _p, ctypes.c_int64, _p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p, _p,
+     _p)
+_sig("akv_stager_create", ctypes.c_int, _p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_p))
+_sig("akv_stage_chunk", ctypes.c_int, _p, _p, ctypes.c_size_t, _p, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+     ctypes.POINTER(_p))
+_sig("akv_stager_use", ctypes.c_int, _p, ctypes.c_int, _p)
+_sig("akv_stager_release", ctypes.c_int, _p, ctypes.c_int, _p)
+_sig("akv_stage_writeback", ctypes.c_int, _p, ctypes.c_int, ctypes.c_size_t, _p, ctypes.c_size_t, _p)
+_sig("akv_stager_destroy", ctypes.c_int, _p)
+
+EXPORTED = [
+    "akv_abi_version", "akv_last_error", "akv_status_string", "akv_error_word_status", "akv_centroids_f16",
+    "akv_plan_slots", "akv_encode_history", "akv_decode_attend", "akv_merge_lse", "akv_stager_create",
+    "akv_stage_chunk", "akv_stager_use", "akv_stager_release", "akv_stage_writeback", "akv_stager_destroy",
+]
+
+
+def _check(status: int) -> int:
+    if status < 0:
+        raise AkvError(status, lib.akv_last_error().decode(errors="replace"))
+    return status
+
+
+def _ptr(x) -> int | None:
+    """Device or host address of a torch tensor / numpy array / int (None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        try:
+            import torch
+            return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _host_i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+@dataclass
+class Tier:
+    """One tier (see ``akv_tier`` in include/akv.h).  k, v, page_table: device tensors or
+    addresses; lens, slot_base: host sequences (kept alive by this object)."""
+    kind: int
+    k: object
+    v: object
+    lens: object
+    slot_base: object = None
+    stride_seq: int = 0
+    stride_head: int = 0
+    stride_token: int = 0
+    paged: bool = False
+    page_table: object = None
+    page_table_stride: int = 0
+    n_pages: int = 0
+    _keep: list = field(default_factory=list, repr=False)
+
+    def c(self) -> AkvTierC:
+        lens = _host_i32(self.lens)
+        slots = _host_i32(self.slot_base) if self.slot_base is not None else None
+        self._keep = [lens, slots]
+        return AkvTierC(self.kind, 1 if self.paged else 0, _ptr(self.k), _ptr(self.v), _ptr(self.page_table),
+                        self.page_table_stride, self.n_pages, self.stride_seq, self.stride_head,
+                        self.stride_token, lens.ctypes.data, None if slots is None else slots.ctypes.data)
+
+
+def abi_version() -> int:
+    return lib.akv_abi_version()
+
+
+def status_string(status: int) -> str:
+    return lib.akv_status_string(status).decode()
+
+
+def error_word_status(word: int) -> int:
+    return lib.akv_error_word_status(int(word))
+
+
+def centroids_f16() -> np.ndarray:
+    out = (ctypes.c_uint16 * 16)()
+    lib.akv_centroids_f16(out)
+    return np.frombuffer(out, dtype=np.uint16).copy()
+
+
+def plan_slots(tier_lens, split_tokens: int):
+    """Standard slot layout.  Returns (tier_slot_base list, seq_slot_base, seq_n_slots, n_slots)."""
+    lens = [_host_i32(t) for t in tier_lens]
+    B = lens[0].size if lens else 0
+    bases = [np.zeros(B, dtype=np.int32) for _ in lens]
+    seq_base = np.zeros(B, dtype=np.int32)
+    seq_n = np.zeros(B, dtype=np.int32)
+    n = ctypes.c_int64(0)
+    lp = (_p * max(1, len(lens)))(*[a.ctypes.data for a in lens])
+    bp = (_p * max(1, len(bases)))(*[a.ctypes.data for a in bases])
+    _check(lib.akv_plan_slots(B, len(lens), lp, split_tokens, bp, seq_base.ctypes.data, seq_n.ctypes.data,
+                              ctypes.byref(n)))
+    return bases, seq_base, seq_n, n.value
+
+
+def akv_encode_history(src: Tier, dst: Tier, B: int, Hkv: int, d: int, err_word=None, stream=None) -> None:
+    s, t = src.c(), dst.c()
+    _check(lib.akv_encode_history(ctypes.byref(s), ctypes.byref(t), B, Hkv, d, _ptr(err_word), _stream(stream)))
+
+
+def akv_decode_attend(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int,
+                      o_part, lse_part, n_slots: int, variant: int = AKV_VARIANT_AUTO, err_word=None,
+                      stream=None) -> None:
+    cs = [t.c() for t in tiers]
+    arr = (AkvTierC * max(1, len(cs)))(*cs)
+    _check(lib.akv_decode_attend(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens,
+                                 _ptr(o_part), _ptr(lse_part), int(n_slots), variant, _ptr(err_word),
+                                 _stream(stream)))
+    del cs
+
+
+def akv_merge_lse(o_part, lse_part, n_slots: int, seq_slot_base, seq_n_slots, B: int, Hq: int, d: int, o, lse,
+                  stream=None) -> None:
+    base = _host_i32(seq_slot_base)
+    cnt = _host_i32(seq_n_slots)
+    _check(lib.akv_merge_lse(_ptr(o_part), _ptr(lse_part), int(n_slots), base.ctypes.data, cnt.ctypes.data, B, Hq,
+                             d, _ptr(o), _ptr(lse), _stream(stream)))
+
+
+class Stager:
+    """Owner of an ``akv_stager`` over a caller-owned device region."""
+
+    def __init__(self, dev_region, region_bytes: int, n_buffers: int):
+        h = _p()
+        _check(lib.akv_stager_create(_ptr(dev_region), region_bytes, n_buffers, ctypes.byref(h)))
+        self._h = h
+        self._region = dev_region  # keep the region alive
+
+    def stage_chunk(self, pinned_src, nbytes: int, copy_stream=None, timeout_ms: int = -1):
+        idx = ctypes.c_int(-1)
+        ptr = _p()
+        _check(lib.akv_stage_chunk(self._h, _ptr(pinned_src), nbytes, _stream(copy_stream), timeout_ms,
+                                   ctypes.byref(idx), ctypes.byref(ptr)))
+        return idx.value, ptr.value
+
+    def use(self, buf: int, consumer_stream=None) -> None:
+        _check(lib.akv_stager_use(self._h, buf, _stream(consumer_stream)))
+
+    def release(self, buf: int, consumer_stream=None) -> None:
+        _check(lib.akv_stager_release(self._h, buf, _stream(consumer_stream)))
+
+    def writeback(self, buf: int, offset: int, pinned_dst, nbytes: int, stream=None) -> None:
+        _check(lib.akv_stage_writeback(self._h, buf, offset, _ptr(pinned_dst), nbytes, _stream(stream)))
+
+    def destroy(self) -> None:
+        if self._h:
+            h, self._h = self._h, None
+            _check(lib.akv_stager_destroy(h))
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass

@@ -1,0 +1,150 @@
+// Internal declarations shared by the libakv translation units: launch-parameter
+// structs (passed by value as __grid_constant__ kernel parameters, so the library needs
+// no device scratch for its per-sequence tables), device helpers for BF16 / tier
+// addressing, and the host-side launchers.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/akv.h"
+
+namespace akv {
+
+// Sequences handled by one launch; larger batches are cut into several launches.
+constexpr int kMaxSeqPerLaunch = 256;
+constexpr int kPageTokens = AKV_PAGE_TOKENS;
+constexpr int kMaxSplitTokens = 1024;
+
+// Device view of one tier (byte pointers; strides in elements for BF16, blocks for CODES4).
+struct TierDev {
+  const uint8_t* k;
+  const uint8_t* v;
+  const int32_t* page_table;
+  int64_t pt_stride;
+  int64_t n_pages;
+  int64_t s_seq, s_head, s_tok;
+  int32_t paged;
+};
+
+// Per-launch sequence table: work item i of the launch belongs to the sequence b with
+// item_base[b] <= i < item_base[b + 1]; b is local to the launch, b0 + b is global.
+struct SeqTable {
+  int32_t n_seq;
+  int32_t b0;
+  int32_t item_base[kMaxSeqPerLaunch + 1];
+  int32_t len[kMaxSeqPerLaunch];
+  int32_t slot_base[kMaxSeqPerLaunch];
+};
+
+struct AttendParams {
+  const uint16_t* q;     // [B][Hq][D] bf16
+  float* o_part;         // [n_slots][Hq][D]
+  float* lse_part;       // [n_slots][Hq]
+  int32_t* err;          // device error word or null
+  TierDev tier;
+  int32_t Hq, Hkv, split_tokens;
+  float scale_log2;      // softmax_scale * log2(e): scores are kept in base-2 units
+  uint16_t centroids[16];
+  SeqTable seq;
+};
+
+struct EncodeParams {
+  TierDev src;           // BF16 tier
+  TierDev dst;           // CODES4 tier (written)
+  int32_t* err;
+  int32_t Hkv;
+  double bound[15];      // decision boundaries (c_j + c_{j+1}) / 2, exact in float64
+  SeqTable seq;          // items are 16-token blocks
+};
+
+struct MergeParams {
+  const float* o_part;
+  const float* lse_part;
+  float* o;
+  float* lse;
+  int32_t Hq;
+  int32_t n_seq, b0;
+  int32_t slot_base[kMaxSeqPerLaunch];
+  int32_t n_slots[kMaxSeqPerLaunch];
+};
+
+// ------------------------------------------------------------------------------------
+// device helpers
+// ------------------------------------------------------------------------------------
+
+__device__ __forceinline__ int find_seq(const SeqTable& st, int item) {
+  int lo = 0, hi = st.n_seq - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (st.item_base[mid] <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// Two packed bf16 -> two floats (exact).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float bf16_to_float(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16); }
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// Physical page of logical page `lp` of global sequence b; out-of-pool ids are flagged
+// and replaced by page 0 so no access leaves the pool.
+__device__ __forceinline__ int64_t tier_page(const TierDev& t, int b, int lp, int32_t* err) {
+  int32_t p = __ldg(t.page_table + (int64_t)b * t.pt_stride + lp);
+  if (p < 0 || (int64_t)p >= t.n_pages) {
+    flag_error(err, AKV_EFLAG_BOUNDS);
+    p = 0;
+  }
+  return p;
+}
+
+// Byte address of the BF16 row of token t (tier-relative), sequence b (global), KV head h.
+__device__ __forceinline__ const uint8_t* bf16_row(const TierDev& t, const uint8_t* base, int b, int h,
+                                                   int tok, int32_t* err) {
+  int64_t e;
+  if (t.paged) {
+    e = tier_page(t, b, tok >> 4, err) * t.s_seq + (int64_t)h * t.s_head + (int64_t)(tok & 15) * t.s_tok;
+  } else {
+    e = (int64_t)b * t.s_seq + (int64_t)h * t.s_head + (int64_t)tok * t.s_tok;
+  }
+  return base + 2 * e;
+}
+
+// Byte address of the CODES4 block holding token t (tier-relative).
+template <int D>
+__device__ __forceinline__ const uint8_t* codes_block(const TierDev& t, const uint8_t* base, int b, int h,
+                                                      int tok, int32_t* err) {
+  constexpr int64_t BB = AKV_CODES4_BLOCK_BYTES(D);
+  int64_t blk;
+  if (t.paged) {
+    blk = tier_page(t, b, tok >> 4, err) * t.s_seq + (int64_t)h * t.s_head;
+  } else {
+    blk = (int64_t)b * t.s_seq + (int64_t)h * t.s_head + (int64_t)(tok >> 4) * t.s_tok;
+  }
+  return base + blk * BB;
+}
+
+// ------------------------------------------------------------------------------------
+// host-side launchers (return cudaGetLastError() of the launch)
+// ------------------------------------------------------------------------------------
+
+cudaError_t launch_encode(const EncodeParams& p, int d, int n_items, cudaStream_t s);
+cudaError_t launch_attend_simt(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
+cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
+cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s);
+
+// host: the binary16 centroid table and its float64 decision boundaries
+const uint16_t* centroid_table_f16();
+const double* centroid_boundaries();
+
+}  // namespace akv

@@ -1,0 +1,467 @@
+// Host side of the libakv C ABI: argument validation (nothing is launched for a refused
+// call), the per-launch sequence tables, the slot planner and the staging ring.
+#include <chrono>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "akv_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+akv_status fail(akv_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+akv_status ok() {
+  g_last_error.clear();
+  return AKV_OK;
+}
+
+akv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(AKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+// Validate a tier for B sequences.  need_slots: check slot ranges against n_slots.
+akv_status check_tier(const akv_tier* t, int idx, int B, int d, int split_tokens, bool need_slots,
+                      int64_t n_slots, int expect_kind) {
+  if (!t) return fail(AKV_ERR_INVALID, "tier %d is null", idx);
+  if (t->kind != AKV_TIER_BF16 && t->kind != AKV_TIER_CODES4)
+    return fail(AKV_ERR_INVALID, "tier %d: unknown kind %d", idx, t->kind);
+  if (expect_kind >= 0 && t->kind != expect_kind)
+    return fail(AKV_ERR_INVALID, "tier %d: kind %d where %d is required", idx, t->kind, expect_kind);
+  if (t->paged != 0 && t->paged != 1) return fail(AKV_ERR_INVALID, "tier %d: paged must be 0 or 1", idx);
+  if (!t->lens) return fail(AKV_ERR_INVALID, "tier %d: lens is null", idx);
+  if (need_slots && !t->slot_base) return fail(AKV_ERR_INVALID, "tier %d: slot_base is null", idx);
+  int64_t max_len = 0;
+  for (int b = 0; b < B; ++b) {
+    if (t->lens[b] < 0) return fail(AKV_ERR_INVALID, "tier %d: lens[%d] = %d < 0", idx, b, t->lens[b]);
+    if (t->lens[b] > max_len) max_len = t->lens[b];
+    if (need_slots && t->lens[b] > 0) {
+      const int64_t ns = ceil_div(t->lens[b], split_tokens);
+      if (t->slot_base[b] < 0 || t->slot_base[b] + ns > n_slots)
+        return fail(AKV_ERR_INVALID, "tier %d: slots [%d, %lld) of sequence %d outside [0, %lld)", idx,
+                    t->slot_base[b], (long long)(t->slot_base[b] + ns), b, (long long)n_slots);
+    }
+  }
+  if (max_len == 0) return AKV_OK;
+  if (!t->k || !t->v) return fail(AKV_ERR_INVALID, "tier %d: k or v is null", idx);
+  if (!aligned(t->k, 16) || !aligned(t->v, 16)) return fail(AKV_ERR_INVALID, "tier %d: k and v must be 16-byte aligned", idx);
+  if (t->stride_seq < 0 || t->stride_head < 0 || t->stride_token < 0)
+    return fail(AKV_ERR_INVALID, "tier %d: negative stride", idx);
+  if (t->kind == AKV_TIER_BF16) {
+    if (t->stride_seq % 8 || t->stride_head % 8 || t->stride_token % 8)
+      return fail(AKV_ERR_INVALID, "tier %d: BF16 strides must be multiples of 8 elements", idx);
+  }
+  if (t->paged) {
+    if (!t->page_table) return fail(AKV_ERR_INVALID, "tier %d: paged tier without page_table", idx);
+    if (t->n_pages <= 0) return fail(AKV_ERR_INVALID, "tier %d: n_pages must be positive", idx);
+    if (t->page_table_stride < ceil_div(max_len, AKV_PAGE_TOKENS))
+      return fail(AKV_ERR_INVALID, "tier %d: page_table_stride %lld < %lld pages needed", idx,
+                  (long long)t->page_table_stride, (long long)ceil_div(max_len, AKV_PAGE_TOKENS));
+  }
+  return AKV_OK;
+}
+
+akv::TierDev tier_dev(const akv_tier* t) {
+  akv::TierDev td;
+  td.k = static_cast<const uint8_t*>(t->k);
+  td.v = static_cast<const uint8_t*>(t->v);
+  td.page_table = t->page_table;
+  td.pt_stride = t->page_table_stride;
+  td.n_pages = t->n_pages;
+  td.s_seq = t->stride_seq;
+  td.s_head = t->stride_head;
+  td.s_tok = t->stride_token;
+  td.paged = t->paged;
+  return td;
+}
+
+// Fill st for sequences [b0, b0 + n) with `items_per_token` granularity; returns items.
+int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, const int32_t* slot_base,
+                       int unit) {
+  st.n_seq = n;
+  st.b0 = b0;
+  int64_t items = 0;
+  for (int i = 0; i < n; ++i) {
+    st.item_base[i] = (int32_t)items;
+    st.len[i] = lens[b0 + i];
+    st.slot_base[i] = slot_base ? slot_base[b0 + i] : 0;
+    items += ceil_div(lens[b0 + i], unit);
+  }
+  st.item_base[n] = (int32_t)items;
+  for (int i = n; i < akv::kMaxSeqPerLaunch; ++i) {
+    st.len[i] = 0;
+    st.slot_base[i] = 0;
+    st.item_base[i + 1] = (int32_t)items;
+  }
+  return items;
+}
+
+}  // namespace
+
+extern "C" {
+
+int akv_abi_version(void) { return AKV_ABI_VERSION; }
+
+const char* akv_last_error(void) { return g_last_error.c_str(); }
+
+const char* akv_status_string(int status) {
+  switch (status) {
+    case AKV_OK: return "ok";
+    case AKV_ERR_INVALID: return "invalid argument";
+    case AKV_ERR_UNSUPPORTED: return "unsupported shape";
+    case AKV_ERR_CUDA: return "CUDA error";
+    case AKV_ERR_NOT_PINNED: return "host memory is not pinned";
+    case AKV_ERR_BUDGET: return "chunk exceeds the staging budget";
+    case AKV_ERR_TIMEOUT: return "staging buffer still in use";
+    case AKV_ERR_NONFINITE: return "non-finite input";
+    case AKV_ERR_RANGE: return "norm out of binary16 range";
+    case AKV_ERR_BOUNDS: return "page id out of bounds";
+    default: return "unknown status";
+  }
+}
+
+akv_status akv_error_word_status(int32_t word) {
+  if (word & AKV_EFLAG_BOUNDS) return AKV_ERR_BOUNDS;
+  if (word & AKV_EFLAG_NONFINITE) return AKV_ERR_NONFINITE;
+  if (word & AKV_EFLAG_RANGE) return AKV_ERR_RANGE;
+  return AKV_OK;
+}
+
+void akv_centroids_f16(uint16_t out[16]) {
+  if (out) std::memcpy(out, akv::centroid_table_f16(), 16 * sizeof(uint16_t));
+}
+
+akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, int split_tokens,
+                          int32_t* const* tier_slot_base, int32_t* seq_slot_base, int32_t* seq_n_slots,
+                          int64_t* n_slots) {
+  if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
+  if (split_tokens <= 0) return fail(AKV_ERR_INVALID, "split_tokens must be positive");
+  if (!n_slots || (B > 0 && (!seq_slot_base || !seq_n_slots)) || (n_tiers > 0 && (!tier_lens || !tier_slot_base)))
+    return fail(AKV_ERR_INVALID, "null output or input array");
+  int64_t slot = 0;
+  for (int b = 0; b < B; ++b) {
+    seq_slot_base[b] = (int32_t)slot;
+    for (int i = 0; i < n_tiers; ++i) {
+      if (!tier_lens[i] || !tier_slot_base[i]) return fail(AKV_ERR_INVALID, "tier %d arrays are null", i);
+      if (tier_lens[i][b] < 0) return fail(AKV_ERR_INVALID, "tier %d: negative length", i);
+      tier_slot_base[i][b] = (int32_t)slot;
+      slot += ceil_div(tier_lens[i][b], split_tokens);
+    }
+    seq_n_slots[b] = (int32_t)(slot - seq_slot_base[b]);
+    if (slot > INT32_MAX) return fail(AKV_ERR_INVALID, "more than 2^31 slots");
+  }
+  *n_slots = slot;
+  return ok();
+}
+
+akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, int Hkv, int d, int32_t* err_word,
+                              akv_stream_t stream) {
+  if (B < 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "B must be >= 0 and Hkv > 0");
+  if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (Hkv > 65535) return fail(AKV_ERR_UNSUPPORTED, "Hkv %d too large", Hkv);
+  akv_status s;
+  if ((s = check_tier(dst, 1, B, d, 16, false, 0, AKV_TIER_CODES4)) != AKV_OK) return s;
+  if (!src) return fail(AKV_ERR_INVALID, "source tier is null");
+  if (src->kind != AKV_TIER_BF16) return fail(AKV_ERR_INVALID, "source tier must be BF16");
+  if (err_word && !aligned(err_word, 4)) return fail(AKV_ERR_INVALID, "err_word must be 4-byte aligned");
+  // the source is addressed with the destination's lengths
+  akv_tier src_view = *src;
+  src_view.lens = dst->lens;
+  src_view.slot_base = nullptr;
+  if ((s = check_tier(&src_view, 0, B, d, 16, false, 0, AKV_TIER_BF16)) != AKV_OK) return s;
+  akv::EncodeParams p;
+  p.src = tier_dev(src);
+  p.dst = tier_dev(dst);
+  p.err = err_word;
+  p.Hkv = Hkv;
+  std::memcpy(p.bound, akv::centroid_boundaries(), sizeof(p.bound));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+    const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+    const int64_t items = fill_seq_table(p.seq, b0, n, dst->lens, nullptr, AKV_PAGE_TOKENS);
+    if (items == 0) continue;
+    if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many blocks in one launch");
+    cudaError_t e = akv::launch_encode(p, d, (int)items, st);
+    if (e != cudaSuccess) return cuda_fail(e, "encode launch");
+  }
+  return ok();
+}
+
+akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
+                             const akv_tier* tiers, int n_tiers, int split_tokens, float* o_part, float* lse_part,
+                             int64_t n_slots, int variant, int32_t* err_word, akv_stream_t stream) {
+  if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(AKV_ERR_INVALID, "Hq must be a positive multiple of Hkv");
+  const int G = Hq / Hkv;
+  if (!supported_group(G)) return fail(AKV_ERR_UNSUPPORTED, "group size %d (supported: 1, 2, 4, 8)", G);
+  if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (Hkv > 65535) return fail(AKV_ERR_UNSUPPORTED, "Hkv %d too large", Hkv);
+  if (split_tokens < 16 || split_tokens > akv::kMaxSplitTokens || split_tokens % 16)
+    return fail(AKV_ERR_UNSUPPORTED, "split_tokens %d (a multiple of 16 in [16, 1024])", split_tokens);
+  if (!std::isfinite(softmax_scale)) return fail(AKV_ERR_INVALID, "softmax_scale is not finite");
+  if (variant != AKV_VARIANT_AUTO && variant != AKV_VARIANT_SIMT && variant != AKV_VARIANT_MMA)
+    return fail(AKV_ERR_INVALID, "unknown variant %d", variant);
+  if (n_slots < 0) return fail(AKV_ERR_INVALID, "n_slots < 0");
+  if (n_tiers > 0 && !tiers) return fail(AKV_ERR_INVALID, "tiers is null");
+  if (err_word && !aligned(err_word, 4)) return fail(AKV_ERR_INVALID, "err_word must be 4-byte aligned");
+  bool any = false;
+  for (int i = 0; i < n_tiers; ++i) {
+    akv_status s = check_tier(&tiers[i], i, B, d, split_tokens, true, n_slots, -1);
+    if (s != AKV_OK) return s;
+    for (int b = 0; b < B; ++b) any |= tiers[i].lens[b] > 0;
+  }
+  if (!any) return ok();
+  if (!q || !aligned(q, 16)) return fail(AKV_ERR_INVALID, "q must be a 16-byte aligned device pointer");
+  if (!o_part || !lse_part) return fail(AKV_ERR_INVALID, "o_part and lse_part must not be null");
+  akv::AttendParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.err = err_word;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.split_tokens = split_tokens;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  std::memcpy(p.centroids, akv::centroid_table_f16(), sizeof(p.centroids));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int i = 0; i < n_tiers; ++i) {
+    p.tier = tier_dev(&tiers[i]);
+    for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+      const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+      const int64_t items = fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens);
+      if (items == 0) continue;
+      if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
+      // AUTO takes the tensor-core path, which measures faster on both tiers
+      cudaError_t e = variant == AKV_VARIANT_SIMT ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
+                                                  : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
+      if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+    }
+  }
+  return ok();
+}
+
+akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_slots, const int32_t* seq_slot_base,
+                         const int32_t* seq_n_slots, int B, int Hq, int d, float* o, float* lse,
+                         akv_stream_t stream) {
+  if (B < 0 || Hq <= 0) return fail(AKV_ERR_INVALID, "B must be >= 0 and Hq > 0");
+  if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (Hq > 65535) return fail(AKV_ERR_UNSUPPORTED, "Hq %d too large", Hq);
+  if (B == 0) return ok();
+  if (!seq_slot_base || !seq_n_slots) return fail(AKV_ERR_INVALID, "slot arrays are null");
+  if (!o || !lse) return fail(AKV_ERR_INVALID, "o and lse must not be null");
+  bool any = false;
+  for (int b = 0; b < B; ++b) {
+    if (seq_n_slots[b] < 0) return fail(AKV_ERR_INVALID, "seq_n_slots[%d] < 0", b);
+    if (seq_n_slots[b] > 0 && (seq_slot_base[b] < 0 || (int64_t)seq_slot_base[b] + seq_n_slots[b] > n_slots))
+      return fail(AKV_ERR_INVALID, "slots of sequence %d outside [0, %lld)", b, (long long)n_slots);
+    any |= seq_n_slots[b] > 0;
+  }
+  if (any && (!o_part || !lse_part)) return fail(AKV_ERR_INVALID, "o_part and lse_part must not be null");
+  akv::MergeParams p;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.o = o;
+  p.lse = lse;
+  p.Hq = Hq;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+    const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+    p.n_seq = n;
+    p.b0 = b0;
+    for (int i = 0; i < akv::kMaxSeqPerLaunch; ++i) {
+      p.slot_base[i] = i < n ? seq_slot_base[b0 + i] : 0;
+      p.n_slots[i] = i < n ? seq_n_slots[b0 + i] : 0;
+    }
+    cudaError_t e = akv::launch_merge(p, d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return ok();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// staging ring
+// ------------------------------------------------------------------------------------
+
+struct akv_stager {
+  struct Buffer {
+    std::vector<cudaEvent_t> pending;  // copies and consumers since the last fill
+    cudaEvent_t ready = nullptr;       // the latest fill's copy
+  };
+  uint8_t* region = nullptr;
+  size_t buf_bytes = 0;
+  int n = 0;
+  int next = 0;
+  std::vector<Buffer> bufs;
+  std::vector<cudaEvent_t> free_events;
+  std::vector<cudaEvent_t> all_events;
+};
+
+namespace {
+
+cudaError_t take_event(akv_stager* st, cudaEvent_t* ev) {
+  if (!st->free_events.empty()) {
+    *ev = st->free_events.back();
+    st->free_events.pop_back();
+    return cudaSuccess;
+  }
+  cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) st->all_events.push_back(*ev);
+  return e;
+}
+
+bool is_pinned(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+}  // namespace
+
+extern "C" {
+
+akv_status akv_stager_create(void* dev_region, size_t region_bytes, int n_buffers, akv_stager** out) {
+  if (!out) return fail(AKV_ERR_INVALID, "out is null");
+  *out = nullptr;
+  if (!dev_region || region_bytes == 0) return fail(AKV_ERR_INVALID, "empty staging region");
+  if (!aligned(dev_region, 256)) return fail(AKV_ERR_INVALID, "staging region must be 256-byte aligned");
+  if (n_buffers < 1 || n_buffers > 64) return fail(AKV_ERR_INVALID, "n_buffers %d outside [1, 64]", n_buffers);
+  auto* st = new akv_stager;
+  st->region = static_cast<uint8_t*>(dev_region);
+  st->buf_bytes = (region_bytes / (size_t)n_buffers) / 256 * 256;
+  st->n = n_buffers;
+  st->bufs.resize(n_buffers);
+  if (st->buf_bytes == 0) {
+    delete st;
+    return fail(AKV_ERR_BUDGET, "region too small for %d buffers", n_buffers);
+  }
+  *out = st;
+  return ok();
+}
+
+akv_status akv_stage_chunk(akv_stager* st, const void* pinned_src, size_t bytes, akv_stream_t copy_stream,
+                           int timeout_ms, int* buf_index, void** dev_ptr) {
+  if (!st || !pinned_src || !buf_index || !dev_ptr) return fail(AKV_ERR_INVALID, "null argument");
+  if (bytes == 0) return fail(AKV_ERR_INVALID, "empty chunk");
+  if (bytes > st->buf_bytes)
+    return fail(AKV_ERR_BUDGET, "chunk of %zu bytes exceeds the %zu-byte staging buffer", bytes, st->buf_bytes);
+  if (!is_pinned(pinned_src) || !is_pinned(static_cast<const uint8_t*>(pinned_src) + bytes - 1))
+    return fail(AKV_ERR_NOT_PINNED, "staging source is not page-locked host memory");
+  const int idx = st->next;
+  akv_stager::Buffer& buf = st->bufs[idx];
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+  if (timeout_ms >= 0) {
+    const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+    for (;;) {
+      bool busy = false;
+      for (cudaEvent_t ev : buf.pending) {
+        cudaError_t q = cudaEventQuery(ev);
+        if (q == cudaErrorNotReady) { busy = true; break; }
+        if (q != cudaSuccess) return cuda_fail(q, "cudaEventQuery");
+      }
+      if (!busy) break;
+      if (std::chrono::steady_clock::now() >= deadline)
+        return fail(AKV_ERR_TIMEOUT, "staging buffer %d still in use after %d ms", idx, timeout_ms);
+      std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
+  }
+  for (cudaEvent_t ev : buf.pending) {
+    cudaError_t e = cudaStreamWaitEvent(cs, ev, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  }
+  // a wait binds to the event's latest record at the time of the call, so the events
+  // can be recycled now
+  for (cudaEvent_t ev : buf.pending) st->free_events.push_back(ev);
+  buf.pending.clear();
+  buf.ready = nullptr;
+  uint8_t* dst = st->region + (size_t)idx * st->buf_bytes;
+  cudaError_t e = cudaMemcpyAsync(dst, pinned_src, bytes, cudaMemcpyHostToDevice, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync H2D");
+  cudaEvent_t ev;
+  if ((e = take_event(st, &ev)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  if ((e = cudaEventRecord(ev, cs)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  buf.pending.push_back(ev);
+  buf.ready = ev;
+  st->next = (idx + 1) % st->n;
+  *buf_index = idx;
+  *dev_ptr = dst;
+  return ok();
+}
+
+akv_status akv_stager_use(akv_stager* st, int buf_index, akv_stream_t consumer_stream) {
+  if (!st || buf_index < 0 || buf_index >= st->n) return fail(AKV_ERR_INVALID, "bad stager or buffer index");
+  akv_stager::Buffer& buf = st->bufs[buf_index];
+  if (!buf.ready) return fail(AKV_ERR_INVALID, "buffer %d has not been filled", buf_index);
+  cudaError_t e = cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(consumer_stream), buf.ready, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  return ok();
+}
+
+akv_status akv_stager_release(akv_stager* st, int buf_index, akv_stream_t consumer_stream) {
+  if (!st || buf_index < 0 || buf_index >= st->n) return fail(AKV_ERR_INVALID, "bad stager or buffer index");
+  cudaEvent_t ev;
+  cudaError_t e = take_event(st, &ev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  if ((e = cudaEventRecord(ev, reinterpret_cast<cudaStream_t>(consumer_stream))) != cudaSuccess) {
+    st->free_events.push_back(ev);
+    return cuda_fail(e, "cudaEventRecord");
+  }
+  st->bufs[buf_index].pending.push_back(ev);
+  return ok();
+}
+
+akv_status akv_stage_writeback(akv_stager* st, int buf_index, size_t offset, void* pinned_dst, size_t bytes,
+                               akv_stream_t stream) {
+  if (!st || buf_index < 0 || buf_index >= st->n || !pinned_dst) return fail(AKV_ERR_INVALID, "bad argument");
+  if (bytes == 0) return ok();
+  if (offset > st->buf_bytes || bytes > st->buf_bytes - offset)
+    return fail(AKV_ERR_BUDGET, "write-back range outside the staging buffer");
+  if (!is_pinned(pinned_dst) || !is_pinned(static_cast<uint8_t*>(pinned_dst) + bytes - 1))
+    return fail(AKV_ERR_NOT_PINNED, "write-back destination is not page-locked host memory");
+  akv_stager::Buffer& buf = st->bufs[buf_index];
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (buf.ready && (e = cudaStreamWaitEvent(s, buf.ready, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  const uint8_t* src = st->region + (size_t)buf_index * st->buf_bytes + offset;
+  if ((e = cudaMemcpyAsync(pinned_dst, src, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyAsync D2H");
+  return akv_stager_release(st, buf_index, stream);
+}
+
+akv_status akv_stager_destroy(akv_stager* st) {
+  if (!st) return ok();
+  akv_status result = AKV_OK;
+  for (auto& b : st->bufs)
+    for (cudaEvent_t ev : b.pending) {
+      cudaError_t e = cudaEventSynchronize(ev);
+      if (e != cudaSuccess && result == AKV_OK) result = cuda_fail(e, "cudaEventSynchronize");
+    }
+  for (cudaEvent_t ev : st->all_events) cudaEventDestroy(ev);
+  delete st;
+  return result == AKV_OK ? ok() : result;
+}
+
+}  // extern "C"

@@ -1,0 +1,195 @@
+"""Device-resident decode workloads driven through the C ABI.
+
+Each class uploads one seeded synthetic workload (``synth``) into device memory in the
+layout the library reads, plans the split slots, and runs one decode step -- every
+tier's split attention followed by the merge -- on a given stream.  Torch provides the
+device memory and streams only.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import akv, synth
+
+
+def to_dev_bits(bits: np.ndarray, device) -> torch.Tensor:
+    """uint16 bit patterns -> device int16 tensor holding the same bits."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device)
+
+
+def tier_lens_slots(tiers):
+    return [t.lens for t in tiers]
+
+
+class DecodeStep:
+    """Partials, outputs and the slot plan shared by every workload."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, d: int, split_tokens: int, scale: float, tiers, device):
+        self.B, self.Hq, self.Hkv, self.d = B, Hq, Hkv, d
+        self.split_tokens, self.scale = split_tokens, scale
+        self.tiers = tiers
+        bases, self.seq_slot_base, self.seq_n_slots, self.n_slots = akv.plan_slots([t.lens for t in tiers], split_tokens)
+        for t, b in zip(tiers, bases):
+            t.slot_base = b
+        self.o_part = torch.empty((max(1, self.n_slots), Hq, d), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty((max(1, self.n_slots), Hq), dtype=torch.float32, device=device)
+        self.o = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def attend(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens,
+                              self.o_part, self.lse_part, self.n_slots, variant, self.err, stream)
+
+    def merge(self, stream=None):
+        akv.akv_merge_lse(self.o_part, self.lse_part, self.n_slots, self.seq_slot_base, self.seq_n_slots, self.B,
+                          self.Hq, self.d, self.o, self.lse, stream)
+
+    def step(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        self.attend(q, variant, stream)
+        self.merge(stream)
+
+    def tier_slots(self, i: int, b: int):
+        """Slot range of tier i, sequence b."""
+        t = self.tiers[i]
+        n = -(-int(t.lens[b]) // self.split_tokens)
+        return int(t.slot_base[b]), n
+
+
+class ExactResident:
+    """Exact BF16 tier, contiguous head-major [B, Hkv, T, d] (the tiny and exact GQA workloads)."""
+
+    def __init__(self, wl: synth.Workload, device, B: int | None = None, T: int | None = None):
+        self.wl = wl
+        B = wl.B if B is None else B
+        T = wl.extra["T"] if T is None else T
+        self.B, self.T = B, T
+        self.q_bits = synth.queries(wl, B=B)
+        ks, vs = [], []
+        for b in range(B):
+            k, v = synth.history_head_major(wl, b, T)
+            ks.append(k)
+            vs.append(v)
+        self.k_bits = np.stack(ks)
+        self.v_bits = np.stack(vs)
+        self.q = to_dev_bits(self.q_bits, device)
+        self.k = to_dev_bits(self.k_bits, device)
+        self.v = to_dev_bits(self.v_bits, device)
+        d, H = wl.d, wl.Hkv
+        tier = akv.Tier(akv.AKV_TIER_BF16, self.k, self.v, lens=np.full(B, T, np.int32),
+                        stride_seq=H * T * d, stride_head=T * d, stride_token=d)
+        self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [tier], device)
+
+    def kv_bytes(self) -> int:
+        return 2 * self.B * self.wl.Hkv * self.T * self.wl.d * 2
+
+
+class HybridResident:
+    """Hybrid tiers of one batch: tokens [0, T - W) compact (contiguous code blocks
+    [B, Hkv, (T - W)/16]), tokens [T - W, T) exact BF16 (a view of the head-major history)."""
+
+    def __init__(self, wl: synth.Workload, device, B: int | None = None, T: int | None = None, W: int | None = None):
+        self.wl = wl
+        B = wl.B if B is None else B
+        T = wl.extra["T"] if T is None else T
+        W = wl.extra["window"] if W is None else W
+        self.B, self.T, self.W = B, T, W
+        d, H = wl.d, wl.Hkv
+        self.q_bits = synth.queries(wl, B=B)
+        ks, vs = [], []
+        for b in range(B):
+            k, v = synth.history_head_major(wl, b, T)
+            ks.append(k)
+            vs.append(v)
+        self.k_bits = np.stack(ks)
+        self.v_bits = np.stack(vs)
+        self.q = to_dev_bits(self.q_bits, device)
+        self.k = to_dev_bits(self.k_bits, device)
+        self.v = to_dev_bits(self.v_bits, device)
+        Tc = T - W
+        nb = -(-Tc // 16)
+        bb = akv.codes4_block_bytes(d)
+        self.kc = torch.empty((B, H, nb, bb), dtype=torch.uint8, device=device)
+        self.vc = torch.empty((B, H, nb, bb), dtype=torch.uint8, device=device)
+        src = akv.Tier(akv.AKV_TIER_BF16, self.k, self.v, lens=np.full(B, Tc, np.int32),
+                       stride_seq=H * T * d, stride_head=T * d, stride_token=d)
+        self.codes_tier = akv.Tier(akv.AKV_TIER_CODES4, self.kc, self.vc, lens=np.full(B, Tc, np.int32),
+                                   stride_seq=H * nb, stride_head=nb, stride_token=1)
+        self.enc_err = torch.zeros(1, dtype=torch.int32, device=device)
+        akv.akv_encode_history(src, self.codes_tier, B, H, d, self.enc_err)
+        off = Tc * d * 2  # bytes: the window starts at token Tc of every (b, h) stream
+        exact = akv.Tier(akv.AKV_TIER_BF16, self.k.data_ptr() + off, self.v.data_ptr() + off,
+                         lens=np.full(B, W, np.int32), stride_seq=H * T * d, stride_head=T * d, stride_token=d)
+        self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [self.codes_tier, exact], device)
+
+    def kv_bytes(self) -> int:
+        d, H = self.wl.d, self.wl.Hkv
+        Tc = self.T - self.W
+        return self.B * H * (2 * self.W * d * 2 + 2 * Tc * (d // 2 + 2))
+
+
+class RaggedPaged:
+    """Ragged paged hybrid batch: per-sequence lengths, 16-token pages drawn from two pools
+    through seeded random page permutations; the newest W tokens exact (BF16 pool
+    [P, Hkv, 16, d]), the rest compact (code-block pool [P, Hkv])."""
+
+    def __init__(self, wl: synth.Workload, device, B: int | None = None, lens=None, W: int | None = None,
+                 key_dist: str = "student_t"):
+        self.wl = wl
+        B = wl.B if B is None else B
+        W = wl.extra["window"] if W is None else W
+        lens = synth.ragged_lengths(wl, B) if lens is None else np.asarray(lens, np.int32)
+        self.B, self.W, self.lens = B, W, lens
+        d, H = wl.d, wl.Hkv
+        self.q_bits = synth.queries(wl, B=B)
+        self.q = to_dev_bits(self.q_bits, device)
+        ex_len = np.minimum(lens, W).astype(np.int32)
+        cp_len = (lens - ex_len).astype(np.int32)
+        ex_pages = -(-ex_len // 16)
+        cp_pages = -(-cp_len // 16)
+        self.ex_table_np = synth.page_tables(ex_pages, synth.page_permutation(wl, "exact", int(ex_pages.sum())))
+        self.cp_table_np = synth.page_tables(cp_pages, synth.page_permutation(wl, "codes", max(1, int(cp_pages.sum()))))
+        n_ex, n_cp = int(ex_pages.sum()), max(1, int(cp_pages.sum()))
+        self.ex_k = torch.zeros((n_ex, H, 16, d), dtype=torch.int16, device=device)
+        self.ex_v = torch.zeros((n_ex, H, 16, d), dtype=torch.int16, device=device)
+        bb = akv.codes4_block_bytes(d)
+        self.cp_k = torch.empty((n_cp, H, bb), dtype=torch.uint8, device=device)
+        self.cp_v = torch.empty((n_cp, H, bb), dtype=torch.uint8, device=device)
+        self.ex_table = torch.from_numpy(self.ex_table_np).to(device)
+        self.cp_table = torch.from_numpy(self.cp_table_np).to(device)
+        self.enc_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.codes_tier = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=cp_len, paged=True,
+                                   page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1],
+                                   n_pages=n_cp, stride_seq=H, stride_head=1)
+        self.exact_tier = akv.Tier(akv.AKV_TIER_BF16, self.ex_k, self.ex_v, lens=ex_len, paged=True,
+                                   page_table=self.ex_table, page_table_stride=self.ex_table_np.shape[1],
+                                   n_pages=n_ex, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
+        self.key_dist = key_dist
+        ex_pool_k = np.zeros((n_ex, H, 16, d), np.uint16)
+        ex_pool_v = np.zeros((n_ex, H, 16, d), np.uint16)
+        for b in range(B):
+            k, v = synth.history_head_major(wl, b, int(lens[b]), key_dist=key_dist)
+            c = int(cp_len[b])
+            synth.scatter_pages(k[:, c:], self.ex_table_np[b], ex_pool_k)
+            synth.scatter_pages(v[:, c:], self.ex_table_np[b], ex_pool_v)
+            if c > 0:
+                # encode the compact part of this sequence into its pages of the code pool
+                ks = to_dev_bits(np.ascontiguousarray(k[:, :c]), device)
+                vs = to_dev_bits(np.ascontiguousarray(v[:, :c]), device)
+                src = akv.Tier(akv.AKV_TIER_BF16, ks, vs, lens=[c], stride_seq=0, stride_head=c * d, stride_token=d)
+                row = self.cp_table[b:b + 1]
+                dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True, page_table=row,
+                               page_table_stride=self.cp_table_np.shape[1], n_pages=n_cp, stride_seq=H,
+                               stride_head=1)
+                akv.akv_encode_history(src, dst, 1, H, d, self.enc_err)
+                torch.cuda.current_stream().synchronize()
+                del ks, vs
+        self.ex_k.copy_(torch.from_numpy(ex_pool_k.view(np.int16)))
+        self.ex_v.copy_(torch.from_numpy(ex_pool_v.view(np.int16)))
+        self.ex_len, self.cp_len = ex_len, cp_len
+        self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [self.codes_tier, self.exact_tier], device)
+
+    def kv_bytes(self) -> int:
+        d, H = self.wl.d, self.wl.Hkv
+        return int(H * (2 * self.ex_len.sum() * d * 2 + 2 * self.cp_len.sum() * (d // 2 + 2)))

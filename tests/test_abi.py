@@ -1,0 +1,138 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol include/akv.h declares,
+and its host-side logic (slot planner, argument validation, centroid table) behaves.
+No call here reaches the GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def akv():
+    from kv_cache_tiering_b200 import build
+    build.build()
+    from kv_cache_tiering_b200 import akv as mod
+    return mod
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(akv_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(akv):
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    for name in syms:
+        assert hasattr(akv.lib, name), name
+        assert ctypes.cast(getattr(akv.lib, name), ctypes.c_void_p).value
+    assert set(akv.EXPORTED) <= set(syms)
+
+
+def test_abi_version_and_status_strings(akv):
+    assert akv.abi_version() == 1
+    assert akv.status_string(0) == "ok"
+    assert akv.status_string(-9) == "page id out of bounds"
+    assert akv.error_word_status(0) == 0
+    assert akv.error_word_status(akv.AKV_EFLAG_RANGE) == akv.AKV_ERR_RANGE
+    assert akv.error_word_status(akv.AKV_EFLAG_RANGE | akv.AKV_EFLAG_BOUNDS) == akv.AKV_ERR_BOUNDS
+
+
+def test_library_table_equals_oracle_table(akv):
+    """The library solves for the Lloyd-Max table with Max's sequential construction; the
+    oracle with Lloyd's iteration.  The binary16 tables must agree bit for bit."""
+    from oracle import lloyd_max
+    assert np.array_equal(akv.centroids_f16(), lloyd_max.centroids_f16_bits())
+
+
+def test_plan_slots(akv):
+    bases, seq_base, seq_n, n = akv.plan_slots([[100, 0, 1024], [30, 5, 0]], 64)
+    assert bases[0].tolist() == [0, 3, 4] and bases[1].tolist() == [2, 3, 20]
+    assert seq_base.tolist() == [0, 3, 4] and seq_n.tolist() == [3, 1, 16] and n == 20
+    with pytest.raises(akv.AkvError) as e:
+        akv.plan_slots([[-1]], 64)
+    assert e.value.status == akv.AKV_ERR_INVALID
+
+
+def _tier(akv, **kw):
+    base = dict(kind=akv.AKV_TIER_BF16, k=0x1000, v=0x2000, lens=[32], slot_base=[0], stride_seq=0,
+                stride_head=4096, stride_token=128)
+    base.update(kw)
+    return akv.Tier(**base)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(d=96), -2),                 # unsupported head dim
+    (dict(Hq=12, Hkv=4), -2),         # G = 3
+    (dict(Hq=10, Hkv=4), -1),         # Hq not a multiple
+    (dict(split_tokens=500), -2),     # not a multiple of 16
+    (dict(split_tokens=2048), -2),    # too large
+    (dict(n_slots=1), -1),            # slots beyond n_slots (32 tokens / 16 = 2 splits)
+    (dict(tier=dict(lens=[-3])), -1),
+    (dict(tier=dict(k=0x1001)), -1),  # misaligned
+    (dict(tier=dict(stride_token=100)), -1),
+    (dict(tier=dict(paged=True, page_table=None, n_pages=4)), -1),
+    (dict(tier=dict(paged=True, page_table=0x3000, n_pages=4, page_table_stride=1)), -1),
+    (dict(q=0x1002), -1),
+    (dict(variant=7), -1),
+])
+def test_attend_refuses_before_launch(akv, args, status):
+    kw = dict(q=0x4000, B=1, Hq=8, Hkv=2, d=128, split_tokens=16, n_slots=4, variant=0)
+    tier_kw = args.pop("tier", {})
+    kw.update(args)
+    t = _tier(akv, **tier_kw)
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_decode_attend(kw["q"], kw["B"], kw["Hq"], kw["Hkv"], kw["d"], 0.1, [t], kw["split_tokens"],
+                              0x5000, 0x6000, kw["n_slots"], kw["variant"], None, 0)
+    assert e.value.status == status
+    assert akv.lib.akv_last_error()
+
+
+def test_empty_work_is_a_no_op(akv):
+    t = _tier(akv, lens=[0], k=0, v=0)
+    akv.akv_decode_attend(0, 1, 8, 2, 128, 0.1, [t], 16, 0, 0, 0, 0, None, 0)
+    akv.akv_merge_lse(0, 0, 0, [0], [0], 0, 8, 128, 0, 0, 0)
+
+
+def test_merge_and_encode_refusals(akv):
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_merge_lse(0x1000, 0x2000, 4, [2], [3], 1, 8, 128, 0x3000, 0x4000, 0)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_merge_lse(0x1000, 0x2000, 4, [0], [3], 1, 8, 80, 0x3000, 0x4000, 0)
+    assert e.value.status == akv.AKV_ERR_UNSUPPORTED
+    src = _tier(akv)
+    dst = _tier(akv, kind=akv.AKV_TIER_CODES4, stride_head=2, stride_token=1)
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_encode_history(dst, dst, 1, 2, 128)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_encode_history(src, dst, 1, 2, 32)
+    assert e.value.status == akv.AKV_ERR_UNSUPPORTED
+
+
+def test_stager_host_refusals(akv):
+    with pytest.raises(akv.AkvError) as e:
+        akv.Stager(0x1000, 1 << 20, 0)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    with pytest.raises(akv.AkvError) as e:
+        akv.Stager(0x1001, 1 << 20, 2)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    st = akv.Stager(0x100000, 1 << 20, 2)  # host bookkeeping only; nothing is touched
+    buf = np.zeros(1 << 20, dtype=np.uint8)
+    with pytest.raises(akv.AkvError) as e:
+        st.stage_chunk(buf, (1 << 19) + 1)
+    assert e.value.status == akv.AKV_ERR_BUDGET
+    with pytest.raises(akv.AkvError) as e:
+        st.use(5)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    st.destroy()
