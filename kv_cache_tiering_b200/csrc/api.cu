@@ -94,9 +94,10 @@ akv::TierDev tier_dev(const akv_tier* t) {
   return td;
 }
 
-// Fill st for sequences [b0, b0 + n) with `items_per_token` granularity; returns items.
+// Fill st for sequences [b0, b0 + n): sequence b owns ceil(len / unit) * mult work
+// items; returns the total.
 int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, const int32_t* slot_base,
-                       int unit) {
+                       int unit, int mult = 1) {
   st.n_seq = n;
   st.b0 = b0;
   int64_t items = 0;
@@ -104,7 +105,7 @@ int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, co
     st.item_base[i] = (int32_t)items;
     st.len[i] = lens[b0 + i];
     st.slot_base[i] = slot_base ? slot_base[b0 + i] : 0;
-    items += ceil_div(lens[b0 + i], unit);
+    items += ceil_div(lens[b0 + i], unit) * mult;
   }
   st.item_base[n] = (int32_t)items;
   for (int i = n; i < akv::kMaxSeqPerLaunch; ++i) {
@@ -247,12 +248,16 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
     p.tier = tier_dev(&tiers[i]);
     for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
       const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
-      const int64_t items = fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens);
+      // the CUDA-core kernels take a (split, KV head) grid; the tensor-core kernels a flat
+      // list of (split, KV head) items
+      const bool simt = variant == AKV_VARIANT_SIMT;
+      const int64_t items =
+          fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv);
       if (items == 0) continue;
       if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
       // AUTO takes the tensor-core path, which measures faster on both tiers
-      cudaError_t e = variant == AKV_VARIANT_SIMT ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
-                                                  : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
+      cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
+                           : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
       if (e != cudaSuccess) return cuda_fail(e, "attend launch");
     }
   }
