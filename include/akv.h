@@ -67,6 +67,7 @@ typedef enum akv_status {
 #define AKV_EFLAG_NONFINITE 0x1
 #define AKV_EFLAG_RANGE 0x2
 #define AKV_EFLAG_BOUNDS 0x4
+#define AKV_EFLAG_TIMEOUT 0x8 /* a kernel's bounded wait for its own copies gave up */
 
 int akv_abi_version(void);
 const char* akv_last_error(void);

@@ -4,6 +4,7 @@
 // addressing, and the host-side launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -39,6 +40,8 @@ struct SeqTable {
 };
 
 struct AttendParams {
+  CUtensorMap tmk, tmv;  // TMA descriptors of a BF16 tier's K and V (tensor-core kernel)
+  int8_t tperm[3];       // TMA dim j+1 takes logical coordinate tperm[j] (0 token, 1 head, 2 seq/page)
   const uint16_t* q;     // [B][Hq][D] bf16
   float* o_part;         // [n_slots][Hq][D]
   float* lse_part;       // [n_slots][Hq]
@@ -141,6 +144,9 @@ __device__ __forceinline__ const uint8_t* codes_block(const TierDev& t, const ui
 cudaError_t launch_encode(const EncodeParams& p, int d, int n_items, cudaStream_t s);
 cudaError_t launch_attend_simt(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
 cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
+// Fill p.tmk / p.tmv for a BF16 tier of B sequences (tokens [0, max_len)): 4-D maps
+// (d, tokens, heads, sequences or pages), 64-element x 16-token boxes, 128-byte swizzle.
+cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int Hkv, int d, int64_t max_len);
 cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s);
 
 // host: the binary16 centroid table and its float64 decision boundaries

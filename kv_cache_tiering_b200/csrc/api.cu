@@ -8,6 +8,11 @@
 #include <thread>
 #include <vector>
 
+#include <algorithm>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
 #include "akv_internal.cuh"
 
 namespace {
@@ -116,7 +121,62 @@ int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, co
   return items;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
 }  // namespace
+
+namespace akv {
+
+// TMA maps of a BF16 tier.  Logical outer coordinates: 0 token (in the page when paged),
+// 1 KV head, 2 sequence (page when paged).  The three outer dims are ordered by byte stride;
+// a dim of extent 1 is placed last with a stride past the others.  Boxes are 64 elements x
+// 16 tokens with 128-byte swizzle; a box that crosses the extent is zero-filled by TMA.
+cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int Hkv, int d, int64_t max_len) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  uint64_t ext[3] = {t->paged ? (uint64_t)AKV_PAGE_TOKENS : (uint64_t)max_len, (uint64_t)Hkv,
+                     t->paged ? (uint64_t)t->n_pages : (uint64_t)B};
+  uint64_t str[3] = {(uint64_t)t->stride_token * 2, (uint64_t)t->stride_head * 2, (uint64_t)t->stride_seq * 2};
+  uint64_t span = 16;
+  for (int i = 0; i < 3; ++i)
+    if (ext[i] > 1) span = std::max(span, str[i] * ext[i]);
+  for (int i = 0; i < 3; ++i) {
+    if (ext[i] > 1 && str[i] == 0) return cudaErrorInvalidValue;  // broadcast strides are not expressible
+    if (ext[i] <= 1) str[i] = span + 16 * (uint64_t)(i + 1);
+  }
+  int order[3] = {0, 1, 2};
+  std::sort(order, order + 3, [&](int a, int b) { return str[a] < str[b]; });
+  cuuint64_t gdim[4] = {(cuuint64_t)d, ext[order[0]], ext[order[1]], ext[order[2]]};
+  cuuint64_t gstr[3] = {str[order[0]], str[order[1]], str[order[2]]};
+  cuuint32_t box[4] = {64, 1, 1, 1};
+  for (int j = 0; j < 3; ++j)
+    if (order[j] == 0) box[j + 1] = AKV_PAGE_TOKENS;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  for (int j = 0; j < 3; ++j) p.tperm[j] = (int8_t)order[j];
+  const void* bases[2] = {t->k, t->v};
+  CUtensorMap* maps[2] = {&p.tmk, &p.tmv};
+  for (int m = 0; m < 2; ++m) {
+    CUresult r = encode(maps[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(bases[m]), gdim, gstr, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace akv
 
 extern "C" {
 
@@ -141,6 +201,7 @@ const char* akv_status_string(int status) {
 }
 
 akv_status akv_error_word_status(int32_t word) {
+  if (word & AKV_EFLAG_TIMEOUT) return AKV_ERR_TIMEOUT;
   if (word & AKV_EFLAG_BOUNDS) return AKV_ERR_BOUNDS;
   if (word & AKV_EFLAG_NONFINITE) return AKV_ERR_NONFINITE;
   if (word & AKV_EFLAG_RANGE) return AKV_ERR_RANGE;
@@ -233,6 +294,7 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
   if (!any) return ok();
   if (!q || !aligned(q, 16)) return fail(AKV_ERR_INVALID, "q must be a 16-byte aligned device pointer");
   if (!o_part || !lse_part) return fail(AKV_ERR_INVALID, "o_part and lse_part must not be null");
+  if (!aligned(o_part, 16)) return fail(AKV_ERR_INVALID, "o_part must be 16-byte aligned");
   akv::AttendParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.o_part = o_part;
@@ -255,6 +317,13 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
           fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv);
       if (items == 0) continue;
       if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
+      if (!simt && tiers[i].kind == AKV_TIER_BF16) {
+        int64_t max_len = 0;
+        for (int b = b0; b < b0 + n; ++b) max_len = std::max<int64_t>(max_len, tiers[i].lens[b]);
+        // global coordinates of the launch's sequences run up to b0 + n
+        if (akv::make_bf16_tensor_maps(p, &tiers[i], b0 + n, Hkv, d, max_len) != cudaSuccess)
+          return fail(AKV_ERR_UNSUPPORTED, "tier %d: cannot describe its layout to the tensor memory accelerator", i);
+      }
       // AUTO takes the tensor-core path, which measures faster on both tiers
       cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
                            : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
@@ -281,6 +350,7 @@ akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_s
     any |= seq_n_slots[b] > 0;
   }
   if (any && (!o_part || !lse_part)) return fail(AKV_ERR_INVALID, "o_part and lse_part must not be null");
+  if (any && !aligned(o_part, 16)) return fail(AKV_ERR_INVALID, "o_part must be 16-byte aligned");
   akv::MergeParams p;
   p.o_part = o_part;
   p.lse_part = lse_part;

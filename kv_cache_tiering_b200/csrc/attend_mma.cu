@@ -8,12 +8,16 @@
 // value written for a split never depends on how many items a call holds or where its
 // tokens live (a staged run equals the resident run bit for bit).
 //
-// Launch.  The grid is persistent: at most one CTA per SM (two groups of NW warps for the
-// compact tier), each owning a contiguous, equal-length range of items (item order is
-// sequence, then KV head, then split, so consecutive items share their query).  Warp w of
-// a group runs chain w of every item of the group back to back through a private ring of
-// NST shared-memory stages filled by cp.async; the ring keeps prefetching across item
-// boundaries while the group merges the finished item.
+// Launch.  The grid is persistent: at most one CTA per SM, each owning a contiguous,
+// equal-length range of items (item order is sequence, then KV head, then split, so
+// consecutive items share their query).  Exact tier: NW = 8 chains per split, warp w runs
+// chain w of every item of the CTA back to back.  Compact tier: one chain per split, each
+// warp owns its own item range.  Every warp streams its steps through a private ring of
+// NST shared-memory stages that keeps prefetching across item boundaries.  Stages are filled by the copy engine, one lane issuing:
+// TMA tiles (cp.async.bulk.tensor, 128-byte swizzle) for BF16 rows, plain bulk copies
+// (cp.async.bulk) for compact code blocks; each stage completes on its own mbarrier.  Every
+// mbarrier wait is bounded: a wait that runs out sets AKV_EFLAG_TIMEOUT and the warp stops
+// computing, drains its copies (again bounded) and leaves.
 //
 // Exact BF16 tier, per step (16 tokens):
 //   S^T (16 rows x 16 tokens) = q . K^T     A = q rows (heads), B = K rows via ldmatrix
@@ -21,7 +25,8 @@
 //                                           accumulator registers
 // The weights P carry a BF16 high part and a BF16 residual: for G <= 4 the residual of
 // head h rides in PV column 4 + h of the same MMA, for G = 8 in a second MMA.
-// Shared-memory tiles are XOR-swizzled in 16-byte chunks so ldmatrix is conflict-free.
+// The TMA swizzle puts 16-byte chunk j of tile row r at chunk j ^ (r & 7) of its 128-byte
+// line, so the ldmatrix row gathers are conflict-free.
 //
 // Compact tier, per step: the same contractions in the rotated basis ("QuantForge V2
 // Walkthrough", section 1: rotate the query instead of the keys) with FP16 operands.  The
@@ -45,12 +50,49 @@ constexpr unsigned kFull = 0xffffffffu;
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
+// ---- mbarriers, TMA and bulk copies
+constexpr uint32_t kWaitLimit = 1u << 22;  // try_wait rounds before a wait gives up
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Bounded wait for phase `parity` of an mbarrier; false when the wait ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -154,7 +196,8 @@ __device__ __forceinline__ void cursor_next(const AttendParams& p, Cursor& c, in
 // online softmax of one step.  sc[j][e] (e < 2): base-2 scores of head g for tokens
 // 8j + 2tq + e, masked with -inf.  Leaves the weights in sc[j][e] and returns the rescale
 // factors of the accumulator columns 2tq, 2tq + 1 (column c holds head c for G = 8 and
-// head c % 4 for G <= 4).  Returns false when no rescale is needed (all factors 1).
+// head c % 4 for G <= 4).  Returns false when no rescale is needed (all factors 1, or the
+// chain's first step, whose accumulators are still zero).
 // ------------------------------------------------------------------------------------
 template <int G>
 __device__ __forceinline__ bool online_softmax(float (&sc)[2][4], float& m_run, float& l_run, float& a_even,
@@ -164,7 +207,7 @@ __device__ __forceinline__ bool online_softmax(float (&sc)[2][4], float& m_run, 
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
   const float m_new = fmaxf(m_run, mx);
-  const bool grow = m_new > m_run;
+  const bool grow = m_new > m_run && m_run != -INFINITY;  // a chain's first step has nothing to rescale
   const float alpha = exp2f(m_run - m_new);  // 0 on a chain's first step (m_run = -inf)
   float s = 0.f;
 #pragma unroll
@@ -263,51 +306,50 @@ __device__ __forceinline__ void warp_fwht(float (&x)[P]) {
 }
 
 // Merge the NW chain states of a finished item (group threads) and write its partials.
-// kRotate: the merged rows are in the rotated basis; rotate back (x H / D) per head.
+// First the G per-head statistics and the NW x G chain factors exp2(m_w - M) / L
+// (/ D as well in the rotated basis) are computed once; then every output is one dot
+// product over chains.  kRotate: the merged rows are in the rotated basis; rotate back.
 template <int D, int G, int NW, bool kRotate>
 __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it, int gi, float* area, float* mws,
-                                           float* lws, float* stage) {
+                                           float* lws, float* fac, float* stage) {
   const int tg = threadIdx.x - gi * NW * 32;  // thread index within the group
   const int warp_in = tg >> 5, lane = threadIdx.x & 31;
-  for (int i = tg; i < G * D; i += NW * 32) {
-    const int h = i / D, dim = i % D;
+  if (tg < G) {
+    const int h = tg;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, mws[w * G + h]);
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) L = fmaf(lws[w * G + h], exp2f(mws[w * G + h] - M), L);
+    const float inv = 1.f / (kRotate ? (float)D * L : L);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) fac[w * G + h] = exp2f(mws[w * G + h] - M) * inv;  // 0 for an empty chain
+    p.lse_part[(size_t)it.slot * p.Hq + it.kvh * G + h] = kLn2 * (M + log2f(L));
+  }
+  group_sync<NW>(gi);
+  for (int i = tg; i < G * D; i += NW * 32) {
+    const int h = i / D, dim = i % D;
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) o = fmaf(area[(w * G + h) * D + dim], exp2f(mws[w * G + h] - M), o);
+    for (int w = 0; w < NW; ++w) o = fmaf(area[(w * G + h) * D + dim], fac[w * G + h], o);
     if constexpr (kRotate) {
       stage[i] = o;
     } else {
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) L = fmaf(lws[w * G + h], exp2f(mws[w * G + h] - M), L);
-      const int hq = it.kvh * G + h;
-      p.o_part[((size_t)it.slot * p.Hq + hq) * D + dim] = o / L;
-      if (dim == 0) p.lse_part[(size_t)it.slot * p.Hq + hq] = kLn2 * (M + log2f(L));
+      p.o_part[((size_t)it.slot * p.Hq + it.kvh * G + h) * D + dim] = o;
     }
   }
   if constexpr (kRotate) {
     group_sync<NW>(gi);
     constexpr int P = D / 32;
     for (int h = warp_in; h < G; h += NW) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, mws[w * G + h]);
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) L = fmaf(lws[w * G + h], exp2f(mws[w * G + h] - M), L);
       float x[P];
 #pragma unroll
       for (int j = 0; j < P; ++j) x[j] = stage[h * D + P * lane + j];
       warp_fwht<P>(x);
-      const float sc = 1.f / ((float)D * L);
-      const int hq = it.kvh * G + h;
-      float* dst = p.o_part + ((size_t)it.slot * p.Hq + hq) * D + P * lane;
+      float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
 #pragma unroll
-      for (int j = 0; j < P; ++j) dst[j] = x[j] * sc;
-      if (lane == 0) p.lse_part[(size_t)it.slot * p.Hq + hq] = kLn2 * (M + log2f(L));
+      for (int j = 0; j < P; ++j) dst[j] = x[j];
     }
   }
 }
@@ -317,68 +359,85 @@ __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it
 // ------------------------------------------------------------------------------------
 template <int D, int G, int NW, int NST>
 struct Bf16Cfg {
-  static constexpr int CH = D / 8;                 // 16-byte chunks per row
-  static constexpr int TILE = 16 * D * 2;          // one 16-token K or V tile
+  static constexpr int HALVES = D / 64;            // 64-element TMA boxes per row
+  static constexpr int BOX = 16 * 128;             // one 16-row x 64-element box
+  static constexpr int TILE = HALVES * BOX;        // one 16-token K or V tile
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int LOADS = 16 * CH / 32;       // cp.async per lane per tile
-  static constexpr int RINGS = NW * NST * STAGE;
+  static constexpr int RINGS = NW * NST * STAGE;   // 1024-byte aligned stages
   static constexpr int AREA = NW * G * D;          // floats
-  static constexpr size_t SMEM = RINGS + (size_t)(AREA + 2 * NW * G) * 4;
+  static constexpr int FLOATS = AREA + 3 * NW * G;  // area, m, l, factors
+  static constexpr int BAR_OFF = RINGS + FLOATS * 4;
+  static constexpr size_t SMEM = BAR_OFF + NW * NST * 8 + 1024;  // + alignment slack
 };
+
+// Byte offset, inside a TMA-swizzled tile, of 16-byte chunk c (of D/8) of row r.
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+  return (uint32_t)((c >> 3) * (16 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
 
 template <int D, int G, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_constant__ AttendParams p) {
   using C = Bf16Cfg<D, G, NW, NST>;
   constexpr int NG = 1;
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  // TMA with 128-byte swizzle wants 1024-byte aligned destinations
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const int gi = 0, w = warp;
   float* area = reinterpret_cast<float*>(smem + C::RINGS);
   float* mws = area + C::AREA;
   float* lws = mws + NW * G;
+  float* fac = lws + NW * G;
   const uint32_t ring_s = smem_u32(smem + warp * NST * C::STAGE);
+  const uint32_t bar_s = smem_u32(smem + C::BAR_OFF) + warp * NST * 8;
 
   int lo, hi;
   cta_range(p.seq.item_base[p.seq.n_seq], lo, hi);
   if (lo >= hi) return;
 
-  // loads of one step into a stage; every row of the step lies in one page
+  if (lane == 0) {
+    for (int j = 0; j < NST; ++j) mbar_init(bar_s + 8 * j, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // lane 0 fills stage st with step s of item it: one TMA box per 64-element half of K and V
   auto load_step = [&](const Item& it, int s, int st) {
-    const int tok0 = it.t0 + 16 * s;
-    const int nv = min(16, it.n - 16 * s);
-    int64_t row0;
-    if (p.tier.paged) {
-      row0 = tier_page(p.tier, it.b, tok0 >> 4, p.err) * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head;
-    } else {
-      row0 = (int64_t)it.b * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head + (int64_t)tok0 * p.tier.s_tok;
-    }
-    const uint8_t* kb = p.tier.k + 2 * row0;
-    const uint8_t* vb = p.tier.v + 2 * row0;
-    const uint32_t st_s = ring_s + st * C::STAGE;
+    if (lane == 0) {
+      int c1, c3;
+      if (p.tier.paged) {
+        c1 = 0;
+        c3 = (int)tier_page(p.tier, it.b, (it.t0 + 16 * s) >> 4, p.err);
+      } else {
+        c1 = it.t0 + 16 * s;
+        c3 = it.b;
+      }
+      const uint32_t bar = bar_s + 8 * st, dst = ring_s + st * C::STAGE;
+      const int lc[3] = {c1, it.kvh, c3};
+      const int x1 = lc[p.tperm[0]], x2 = lc[p.tperm[1]], x3 = lc[p.tperm[2]];
+      fence_proxy_async();
+      mbar_expect_tx(bar, C::STAGE);
 #pragma unroll
-    for (int i = 0; i < C::LOADS; ++i) {
-      const int idx = i * 32 + lane;
-      const int r = idx / C::CH, c = idx % C::CH;
-      const int64_t e = (int64_t)(r < nv ? r : 0) * p.tier.s_tok + 8 * c;
-      const uint32_t off = (uint32_t)(r * D * 2 + ((c ^ (r & 7)) << 4));
-      const int bytes = r < nv ? 16 : 0;
-      cp_async16(st_s + off, kb + 2 * e, bytes);
-      cp_async16(st_s + C::TILE + off, vb + 2 * e, bytes);
+      for (int hv = 0; hv < C::HALVES; ++hv) {
+        tma_load_4d(dst + hv * C::BOX, &p.tmk, 64 * hv, x1, x2, x3, bar);
+        tma_load_4d(dst + C::TILE + hv * C::BOX, &p.tmv, 64 * hv, x1, x2, x3, bar);
+      }
     }
   };
 
   Cursor ld;
   ld.item = lo + gi;
   ld.step = w;
-  if (ld.item < hi) ld.info = item_at(p, ld.item);
+  ld.info = item_at(p, ld.item);
   cursor_settle<NG>(p, ld, hi, w);
+  int issued = 0;
 #pragma unroll
   for (int j = 0; j < NST; ++j) {
     if (ld.item < hi) {
       load_step(ld.info, ld.step, j);
       cursor_next<NW, NG>(p, ld, hi, w);
+      ++issued;
     }
-    cp_async_commit();
   }
 
   int dim_of[D / 16][2];
@@ -390,6 +449,8 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
   uint32_t qa[D / 16][4];
   int q_pair = -1;
   int stage = 0;
+  uint32_t phases = 0;  // bit j: parity of stage j's next completion
+  bool ok = true;
 
   for (int item = lo + gi; item < hi; item += NG) {
     const Item it = item_at(p, item);
@@ -414,79 +475,103 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
     float m_run = -INFINITY, l_run = 0.f;
 
     for (int s = w; 16 * s < it.n; s += NW) {
-      cp_async_wait<NST - 1>();
-      __syncwarp();
-      const int nv = min(16, it.n - 16 * s);
-      const uint32_t kt = ring_s + stage * C::STAGE, vt = kt + C::TILE;
-      float sc[2][4];
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[j][e] = 0.f;
-#pragma unroll
-      for (int kc = 0; kc < D / 16; ++kc) {
-        const int mi = lane >> 3, r = (mi >> 1) * 8 + (lane & 7), c = 2 * kc + (mi & 1);
-        uint32_t b[4];
-        ldsm_x4(b, kt + r * D * 2 + ((c ^ (r & 7)) << 4));
-        mma_bf16(sc[0], qa[kc], b[0], b[1]);
-        mma_bf16(sc[1], qa[kc], b[2], b[3]);
-      }
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) sc[j][e] *= p.scale_log2;
-      if (nv < 16) {
+      if (ok) ok = __all_sync(kFull, mbar_wait(bar_s + 8 * stage, (phases >> stage) & 1u));  // warp-uniform
+      phases ^= 1u << stage;
+      --issued;
+      if (ok) {
+        const int nv = min(16, it.n - 16 * s);
+        const uint32_t kt = ring_s + stage * C::STAGE, vt = kt + C::TILE;
+        uint8_t* vt_g = smem + warp * NST * C::STAGE + stage * C::STAGE + C::TILE;
+        if (nv < 16) {  // rows past the split may hold anything: clear them in V
+          for (int i = lane; i < (16 - nv) * C::HALVES * 8; i += 32) {
+            const int r = nv + i / (C::HALVES * 8), rem = i % (C::HALVES * 8);
+            *reinterpret_cast<uint4*>(vt_g + (rem >> 3) * C::BOX + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+          }
+          __syncwarp();
+        }
+        float sc[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
-          for (int e = 0; e < 2; ++e)
-            if (8 * j + 2 * tq + e >= nv) sc[j][e] = -INFINITY;
-      }
-      float a_even, a_odd;
-      if (online_softmax<G>(sc, m_run, l_run, a_even, a_odd)) {
+          for (int e = 0; e < 4; ++e) sc[j][e] = 0.f;
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) {
+          const int mi = lane >> 3, r = (mi >> 1) * 8 + (lane & 7), c = 2 * kc + (mi & 1);
+          uint32_t b[4];
+          ldsm_x4(b, kt + tile_off(r, c));
+          mma_bf16(sc[0], qa[kc], b[0], b[1]);
+          mma_bf16(sc[1], qa[kc], b[2], b[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) sc[j][e] *= p.scale_log2;
+        if (nv < 16) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              if (8 * j + 2 * tq + e >= nv) sc[j][e] = -INFINITY;
+        }
+        float a_even, a_odd;
+        if (online_softmax<G>(sc, m_run, l_run, a_even, a_odd)) {
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            acc[mt][0] *= a_even; acc[mt][1] *= a_odd;
+            acc[mt][2] *= a_even; acc[mt][3] *= a_odd;
+          }
+        }
+        const float wts[2][2] = {{sc[0][0], sc[0][1]}, {sc[1][0], sc[1][1]}};
+        uint32_t pb[2], pl[2];
+        p_fragments<G, true>(wts, pb, pl);
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
-          acc[mt][0] *= a_even; acc[mt][1] *= a_odd;
-          acc[mt][2] *= a_even; acc[mt][3] *= a_odd;
+          const int mi = lane >> 3, r = (mi >> 1) * 8 + (lane & 7), c = 2 * mt + (mi & 1);
+          uint32_t a[4];
+          ldsm_x4_t(a, vt + tile_off(r, c));
+          mma_bf16(acc[mt], a, pb[0], pb[1]);
+          if constexpr (G > 4) mma_bf16(acc[mt], a, pl[0], pl[1]);
+        }
+        __syncwarp();
+        if (ld.item < hi) {
+          load_step(ld.info, ld.step, stage);
+          cursor_next<NW, NG>(p, ld, hi, w);
+          ++issued;
         }
       }
-      const float wts[2][2] = {{sc[0][0], sc[0][1]}, {sc[1][0], sc[1][1]}};
-      uint32_t pb[2], pl[2];
-      p_fragments<G, true>(wts, pb, pl);
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        const int mi = lane >> 3, r = (mi >> 1) * 8 + (lane & 7), c = 2 * mt + (mi & 1);
-        uint32_t a[4];
-        ldsm_x4_t(a, vt + r * D * 2 + ((c ^ (r & 7)) << 4));
-        mma_bf16(acc[mt], a, pb[0], pb[1]);
-        if constexpr (G > 4) mma_bf16(acc[mt], a, pl[0], pl[1]);
-      }
-      __syncwarp();
-      if (ld.item < hi) {
-        load_step(ld.info, ld.step, stage);
-        cursor_next<NW, NG>(p, ld, hi, w);
-      }
-      cp_async_commit();
       stage = stage + 1 == NST ? 0 : stage + 1;
     }
     chain_to_smem<D, G>(acc, m_run, l_run, area + w * G * D, mws + w * G, lws + w * G, dim_of);
     group_sync<NW>(gi);
-    merge_item<D, G, NW, false>(p, it, gi, area, mws, lws, nullptr);
+    merge_item<D, G, NW, false>(p, it, gi, area, mws, lws, fac, nullptr);
     group_sync<NW>(gi);
   }
-  cp_async_wait<0>();
+  if (!ok) {
+    // a wait ran out: record it, then give the copies still in flight a bounded chance
+    // to land before the CTA's shared memory goes away
+    if (lane == 0) flag_error(p.err, AKV_EFLAG_TIMEOUT);
+    for (; issued > 0; --issued) {
+      mbar_wait(bar_s + 8 * stage, (phases >> stage) & 1u);
+      phases ^= 1u << stage;
+      stage = stage + 1 == NST ? 0 : stage + 1;
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------
-// compact tier (CODES4)
+// compact tier (CODES4): one warp per split
 // ------------------------------------------------------------------------------------
-// Shared memory: the lookup table lut[256][32] (entry b for lane l: the half pair
-// (c[b & 15], c[b >> 4]); one copy per lane keeps the gathers conflict-free), then per
-// group: the query words qw[G][D] (FP16 high/residual pairs of H q / 2^e), qscale[8],
-// the merge area and staging rows; then one ring per warp.  A stage holds one 16-token
-// block of K (code rows unpadded, then 16 scales) and of V (code rows padded to VROW
-// bytes so the four token lanes' reads fall in different banks, then 16 scales).
-template <int D, int G, int NW, int NG, int NST>
+// Every split of the compact tier is one chain: a single warp runs all of its 16-token
+// steps in order, so the split needs no cross-warp merge.  The grid is persistent (one CTA
+// of NWARP warps per SM) and every warp owns an equal contiguous range of items.
+// Shared memory: the lookup table, 256 rows of 256 bytes (entry b for lane l at byte
+// 256 b + 4 l: the half pair (c[b & 15], c[b >> 4]); one copy per lane keeps the gathers
+// conflict-free, and the row stride lets one byte permute build the address); then per
+// warp a scratch of G x D words (query rotation, output rotation) and a ring of NST
+// stages.  A stage holds one 16-token block of K (its own layout: code rows, then 16
+// scales) and of V (code rows padded to VROW bytes so the four token lanes' reads fall in
+// different banks, then 16 scales), filled by cp.async.
+template <int D, int G, int NWARP, int NST>
 struct CodesCfg {
   static constexpr int ROWB = D / 2;
   static constexpr int VROW = ROWB + 16;
@@ -496,103 +581,108 @@ struct CodesCfg {
   static constexpr int VS_OFF = V_OFF + 16 * VROW;
   static constexpr int STAGE = VS_OFF + 32;
   static constexpr int BLOCK = AKV_CODES4_BLOCK_BYTES(D);
-  static constexpr int CHUNKS = BLOCK / 16;
-  static constexpr int LUT = 256 * 32 * 4;
-  // per-group floats: query words G*D, qscale 8, merge area NW*G*D, m and l 2*NW*G, stage G*D
-  static constexpr int GROUP = G * D + 8 + NW * G * D + 2 * NW * G + G * D;
-  static constexpr int RING_OFF = LUT + NG * GROUP * 4;
-  static constexpr size_t SMEM = (size_t)RING_OFF + (size_t)NG * NW * NST * STAGE;
+  static constexpr int LUT = 256 * 256;
+  static constexpr int SCRATCH = (G * D + 16) * 4;  // words, plus per-head scales
+  static constexpr int PER_WARP = SCRATCH + NST * STAGE;
+  static constexpr size_t SMEM = (size_t)LUT + (size_t)NWARP * PER_WARP;
 };
 
-template <int D, int G, int NW, int NG, int NST>
-__global__ void __launch_bounds__(NW * NG * 32, 1) attend_codes_mma(const __grid_constant__ AttendParams p) {
-  using C = CodesCfg<D, G, NW, NG, NST>;
+template <int D, int G, int NWARP, int NST>
+__global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_constant__ AttendParams p) {
+  using C = CodesCfg<D, G, NWARP, NST>;
   constexpr int DPT = D / 8;                      // value dims per lane group
   constexpr int KB = D / 8;                       // key code bytes per lane
   constexpr int NWD = DPT / 8 > 0 ? DPT / 8 : 1;  // value code words per token per lane
+  constexpr int P = D / 32;                       // coordinates per lane in a warp-wide row
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const int gi = warp / NW, w = warp % NW;
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  float* gbase = reinterpret_cast<float*>(smem + C::LUT) + gi * C::GROUP;
-  uint32_t* qwords = reinterpret_cast<uint32_t*>(gbase);   // [G][D]
-  float* qscale = gbase + G * D;                            // [8]
-  float* area = qscale + 8;                                 // [NW][G][D]
-  float* mws = area + NW * G * D;
-  float* lws = mws + NW * G;
-  float* stagef = lws + NW * G;                             // [G][D]
-  uint8_t* ring = smem + C::RING_OFF + (size_t)warp * NST * C::STAGE;
+  uint8_t* wbase = smem + C::LUT + (size_t)warp * C::PER_WARP;
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(wbase);   // [G][D] words
+  float* scratchf = reinterpret_cast<float*>(wbase);
+  float* hscale = reinterpret_cast<float*>(wbase) + G * D;  // [G]
+  uint8_t* ring = wbase + C::SCRATCH;
   const uint32_t ring_s = smem_u32(ring);
 
-  for (int i = threadIdx.x; i < 256 * 32; i += NW * NG * 32) {
-    const int byte = i >> 5;
-    lut[i] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
+  for (int i = threadIdx.x; i < 256 * 32; i += NWARP * 32) {
+    const int byte = i >> 5, l = i & 31;
+    lut[byte * 64 + l] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
   }
   __syncthreads();
 
-  int lo, hi;
-  cta_range(p.seq.item_base[p.seq.n_seq], lo, hi);
-  if (lo + gi >= hi) return;  // a group without items (no block-wide barrier follows)
+  // this warp's item range: an equal share of all items, in item order
+  const int total = p.seq.item_base[p.seq.n_seq];
+  const int nw = (int)gridDim.x * NWARP, gw = (int)blockIdx.x * NWARP + warp;
+  const int q0 = total / nw, r0 = total % nw;
+  const int lo = gw * q0 + min(gw, r0), hi = lo + q0 + (gw < r0 ? 1 : 0);
+  if (lo >= hi) return;
 
+  // stage fill through cp.async 16-byte chunks: lane l copies code chunks l and l + 32 of K
+  // (the block's own layout) and of V (into the padded rows); lanes 0 and 1 also copy the
+  // two scale chunks of each
+  constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per code row
+  constexpr bool kTwo = C::ROWB > 32;
+  const uint32_t kd0 = C::K_OFF + 16 * lane, kd1 = kd0 + 16 * 32;
+  const uint32_t vd0 = C::V_OFF + (lane / CPR) * C::VROW + 16 * (lane % CPR);
+  const uint32_t vd1 = C::V_OFF + ((lane + 32) / CPR) * C::VROW + 16 * ((lane + 32) % CPR);
   auto load_step = [&](const Item& it, int s, int st) {
     const int tok0 = it.t0 + 16 * s;
-    const uint8_t* kb = codes_block<D>(p.tier, p.tier.k, it.b, it.kvh, tok0, p.err);
-    const uint8_t* vb = codes_block<D>(p.tier, p.tier.v, it.b, it.kvh, tok0, p.err);
-    const uint32_t st_s = ring_s + st * C::STAGE;
-#pragma unroll
-    for (int i0 = 0; i0 < C::CHUNKS; i0 += 32) {
-      const int i = i0 + lane;
-      if (i < C::CHUNKS) {
-        cp_async16(st_s + C::K_OFF + 16 * i, kb + 16 * i, 16);
-        uint32_t voff;
-        if (i < C::ROWB) {
-          const int r = i / (C::ROWB / 16), c = i % (C::ROWB / 16);
-          voff = C::V_OFF + r * C::VROW + 16 * c;
-        } else {
-          voff = C::VS_OFF + 16 * (i - C::ROWB);
-        }
-        cp_async16(st_s + voff, vb + 16 * i, 16);
-      }
+    int64_t blk;
+    if (p.tier.paged) {
+      blk = tier_page(p.tier, it.b, tok0 >> 4, p.err) * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head;
+    } else {
+      blk = (int64_t)it.b * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head + (int64_t)(tok0 >> 4) * p.tier.s_tok;
+    }
+    const uint8_t* kb = p.tier.k + blk * C::BLOCK + 16 * lane;
+    const uint8_t* vb = p.tier.v + blk * C::BLOCK + 16 * lane;
+    const uint32_t dst = ring_s + st * C::STAGE;
+    cp_async16(dst + kd0, kb);
+    cp_async16(dst + vd0, vb);
+    if constexpr (kTwo) {
+      cp_async16(dst + kd1, kb + 16 * 32);
+      cp_async16(dst + vd1, vb + 16 * 32);
+    }
+    if (lane < 2) {
+      cp_async16(dst + C::KS_OFF + 16 * lane, kb + 16 * C::ROWB);
+      cp_async16(dst + C::VS_OFF + 16 * lane, vb + 16 * C::ROWB);
     }
   };
 
+  // cursor over (item, step): all steps of each item in order
   Cursor ld;
-  ld.item = lo + gi;
-  ld.step = w;
+  ld.item = lo;
+  ld.step = 0;
   ld.info = item_at(p, ld.item);
-  cursor_settle<NG>(p, ld, hi, w);
 #pragma unroll
   for (int j = 0; j < NST; ++j) {
     if (ld.item < hi) {
       load_step(ld.info, ld.step, j);
-      cursor_next<NW, NG>(p, ld, hi, w);
+      cursor_next<1, 1>(p, ld, hi, 0);
     }
     cp_async_commit();
   }
 
-  const uint32_t* my_lut = lut + lane;
+  // table address of byte `byte` of `word` for this lane: (word.byte << 8) | (lane << 2)
+  const uint32_t lane4 = (uint32_t)lane << 2;
   auto lookup = [&](uint32_t word, int byte) -> uint32_t {
-    return my_lut[__byte_perm(word, 0, 0x4440 + byte) * 32];
+    const uint32_t addr = __byte_perm(word, lane4, 0x5504 | (byte << 4));
+    return *reinterpret_cast<const uint32_t*>(smem + addr);
   };
 
-  int dim_of[D / 16][2];
-#pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) {
-    dim_of[mt][0] = DPT * g + mt;
-    dim_of[mt][1] = DPT * g + DPT / 2 + mt;
-  }
   uint32_t qa[D / 16][4];
   float kfac = 0.f;
   int q_pair = -1;
   int stage = 0;
 
-  for (int item = lo + gi; item < hi; item += NG) {
+  for (int item = lo; item < hi; ++item) {
     const Item it = item_at(p, item);
     if (it.pair != q_pair) {
       q_pair = it.pair;
-      // warp h rotates head h: H q by shuffles, a power-of-two scale to [0.5, 1), FP16 hi/lo
-      constexpr int P = D / 32;
-      for (int h = w; h < G; h += NW) {
+      // rotate each head: H q by shuffles, a power-of-two scale to [0.5, 1), then the
+      // FP16 (high, residual) words of dims (P*lane + j, P*lane + j + 1) into the scratch
+      __syncwarp();
+#pragma unroll 1
+      for (int h = 0; h < G; ++h) {
         const uint16_t* qrow = p.q + ((size_t)it.b * p.Hq + (size_t)it.kvh * G + h) * D + P * lane;
         float x[P];
 #pragma unroll
@@ -611,17 +701,16 @@ __global__ void __launch_bounds__(NW * NG * 32, 1) attend_codes_mma(const __grid
           const float x0 = x[j] * inv, x1 = x[j + 1] * inv;
           const uint32_t hw = pack_f16(x0, x1);
           const float2 hv = unpack_f16(hw);
-          // (high, residual) words of dims (P*lane + j, P*lane + j + 1)
-          qwords[h * D + P * lane + j] = hw;
-          qwords[h * D + P * lane + j + 1] = pack_f16(x0 - hv.x, x1 - hv.y);
+          scratch[h * D + P * lane + j] = hw;
+          scratch[h * D + P * lane + j + 1] = pack_f16(x0 - hv.x, x1 - hv.y);
         }
-        if (lane == 0) qscale[h] = ldexpf(1.f, e);
+        if (lane == 0) hscale[h] = ldexpf(1.f, e);
       }
-      group_sync<NW>(gi);
+      __syncwarp();
       // lane (g, tq), step kc covers dims 2*KB*tq + 4kc + {0,1,2,3}: rows g = high parts,
       // rows g + 8 = residuals
       const int h = g < G ? g : 0;
-      const uint32_t* qrow = qwords + h * D + 2 * KB * tq;
+      const uint32_t* qrow = scratch + h * D + 2 * KB * tq;
 #pragma unroll
       for (int kc = 0; kc < D / 16; ++kc) {
         qa[kc][0] = g < G ? qrow[4 * kc] : 0u;       // high, dims 4kc, 4kc+1
@@ -629,8 +718,8 @@ __global__ void __launch_bounds__(NW * NG * 32, 1) attend_codes_mma(const __grid
         qa[kc][2] = g < G ? qrow[4 * kc + 2] : 0u;   // high, dims 4kc+2, 4kc+3
         qa[kc][3] = g < G ? qrow[4 * kc + 3] : 0u;   // residual
       }
-      kfac = p.scale_log2 / (float)D * qscale[h];
-      group_sync<NW>(gi);
+      kfac = p.scale_log2 / (float)D * hscale[h];
+      __syncwarp();
     }
 
     float acc[D / 16][4];
@@ -640,32 +729,34 @@ __global__ void __launch_bounds__(NW * NG * 32, 1) attend_codes_mma(const __grid
       for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;
 
-    for (int s = w; 16 * s < it.n; s += NW) {
+    for (int s = 0; 16 * s < it.n; ++s) {
       cp_async_wait<NST - 1>();
       __syncwarp();
       const int nv = min(16, it.n - 16 * s);
       const uint8_t* sk = ring + stage * C::STAGE;
       // ---- S^T = (H q) K_hat^T: B fragments straight from the code bytes
       float sc[2][4];
+      uint32_t wk[2][KB / 4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) sc[j][e] = 0.f;
-        uint32_t wk[KB / 4];
         const uint8_t* row = sk + C::K_OFF + (8 * j + g) * C::ROWB + KB * tq;
         if constexpr (KB == 16) {
           const uint4 v = *reinterpret_cast<const uint4*>(row);
-          wk[0] = v.x; wk[1] = v.y; wk[2] = v.z; wk[3] = v.w;
+          wk[j][0] = v.x; wk[j][1] = v.y; wk[j][2] = v.z; wk[j][3] = v.w;
         } else {
           const uint2 v = *reinterpret_cast<const uint2*>(row);
-          wk[0] = v.x; wk[1] = v.y;
-        }
-#pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc) {
-          const uint32_t wd = wk[kc >> 1];
-          mma_f16(sc[j], qa[kc], lookup(wd, 2 * (kc & 1)), lookup(wd, 2 * (kc & 1) + 1));
+          wk[j][0] = v.x; wk[j][1] = v.y;
         }
       }
+#pragma unroll
+      for (int kc = 0; kc < D / 16; ++kc)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t wd = wk[j][kc >> 1];
+          mma_f16(sc[j], qa[kc], lookup(wd, 2 * (kc & 1)), lookup(wd, 2 * (kc & 1) + 1));
+        }
       float ksc[2][2], vsc[2][2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -746,15 +837,51 @@ __global__ void __launch_bounds__(NW * NG * 32, 1) attend_codes_mma(const __grid
       __syncwarp();
       if (ld.item < hi) {
         load_step(ld.info, ld.step, stage);
-        cursor_next<NW, NG>(p, ld, hi, w);
+        cursor_next<1, 1>(p, ld, hi, 0);
       }
       cp_async_commit();
       stage = stage + 1 == NST ? 0 : stage + 1;
     }
-    chain_to_smem<D, G>(acc, m_run, l_run, area + w * G * D, mws + w * G, lws + w * G, dim_of);
-    group_sync<NW>(gi);
-    merge_item<D, G, NW, true>(p, it, gi, area, mws, lws, stagef);
-    group_sync<NW>(gi);
+
+    // ---- epilogue: O = H (acc / l) / D per head, LSE = ln 2 (m + log2 l)
+    l_run += __shfl_xor_sync(kFull, l_run, 1);
+    l_run += __shfl_xor_sync(kFull, l_run, 2);
+    if (tq == 0 && g < G)
+      p.lse_part[(size_t)it.slot * p.Hq + it.kvh * G + g] = kLn2 * (m_run + log2f(l_run));
+    const float inv_l = 1.f / ((float)D * l_run);
+    constexpr int HM = G <= 4 ? 3 : 7;
+    const float f_even = __shfl_sync(kFull, inv_l, ((2 * tq) & HM) * 4);
+    const float f_odd = __shfl_sync(kFull, inv_l, ((2 * tq + 1) & HM) * 4);
+    if constexpr (G <= 4) {  // fold the residual columns 4..7 into heads 0..3
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] += __shfl_xor_sync(kFull, acc[mt][e], 2);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = 2 * tq + (e & 1);
+        const int dim = DPT * g + ((e >> 1) ? DPT / 2 : 0) + mt;
+        if (h < G) scratchf[h * D + dim] = acc[mt][e] * ((e & 1) ? f_odd : f_even);
+      }
+    __syncwarp();
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+      float x[P];
+#pragma unroll
+      for (int j = 0; j < P; ++j) x[j] = scratchf[h * D + P * lane + j];
+      warp_fwht<P>(x);
+      float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
+      if constexpr (P == 4) {
+        *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+      } else {
+        *reinterpret_cast<float2*>(dst) = make_float2(x[0], x[1]);
+      }
+    }
+    __syncwarp();
   }
   cp_async_wait<0>();
 }
@@ -782,17 +909,16 @@ cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s) {
 
 template <int D, int G>
 cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
-  constexpr int NW = 8;
-  constexpr int NG = G <= 4 ? 2 : 1;
-  constexpr int NST = 4;
-  using C = CodesCfg<D, G, NW, NG, NST>;
-  auto k = attend_codes_mma<D, G, NW, NG, NST>;
+  constexpr int NWARP = G <= 4 ? 16 : 8;
+  constexpr int NST = 3;
+  using C = CodesCfg<D, G, NWARP, NST>;
+  auto k = attend_codes_mma<D, G, NWARP, NST>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
-  const int want = (n_items + NG - 1) / NG;
+  const int want = (n_items + NWARP - 1) / NWARP;
   const int grid = want < sms ? want : sms;
-  k<<<grid, NW * NG * 32, C::SMEM, s>>>(p);
+  k<<<grid, NWARP * 32, C::SMEM, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -1,40 +1,117 @@
 // Exact log-sum-exp merge of split partials ("Context beyond VRAM", section "What I
-// built": the tiers are merged with exact attention arithmetic).  One CTA of D threads
-// per (sequence, query head); thread i owns output coordinate i.  The partials of a
-// sequence are read in increasing slot order, so the result is deterministic.
+// built": the tiers are merged with exact attention arithmetic).
+//
+// One CTA of 256 threads per (sequence, query head).  The slots of the sequence are taken
+// in chunks of up to kChunk:
+//   1. M = max of the chunk's LSE values joined with the running maximum;
+//   2. w_s = exp(LSE_s - M) into shared memory, their sum L;
+//   3. warp w accumulates slots w, w + 8, ... of the chunk, lane l owning coordinates
+//      [P*l, P*l + P) (coalesced rows), and the eight warp sums are added in warp order.
+// Partial sums from an earlier chunk are rescaled by exp(M_old - M_new).  Every sum is taken
+// in a fixed order, so the result is deterministic.
 #include "akv_internal.cuh"
 
 namespace akv {
 namespace {
 
+constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kChunk = 1024;
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = red[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) s += red[w];
+  return s;
+}
+
 template <int D>
-__global__ void __launch_bounds__(D) merge_kernel(const __grid_constant__ MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ MergeParams p) {
+  constexpr int P = D / 32;  // coordinates per lane
+  __shared__ float wsh[kChunk];
+  __shared__ float red[kMergeWarps];
+  __shared__ float acc_sh[kMergeWarps][D];
   const int bl = blockIdx.x, h = blockIdx.y;
   const int b = p.b0 + bl;
   const int base = p.slot_base[bl], n = p.n_slots[bl];
-  const int i = threadIdx.x;
-  float m = -INFINITY;
-  for (int s = 0; s < n; ++s) m = fmaxf(m, __ldg(p.lse_part + (size_t)(base + s) * p.Hq + h));
-  float o = 0.f, l = 0.f;
-  if (m != -INFINITY) {
-    for (int s = 0; s < n; ++s) {
-      const float ls = __ldg(p.lse_part + (size_t)(base + s) * p.Hq + h);
-      const float w = expf(ls - m);  // exp(-inf) = 0 for an empty partial
-      l += w;
-      o = fmaf(w, __ldg(p.o_part + ((size_t)(base + s) * p.Hq + h) * D + i), o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  float M = -INFINITY, L = 0.f;
+  float acc[P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) acc[j] = 0.f;
+
+  for (int c0 = 0; c0 < n; c0 += kChunk) {
+    const int cn = min(kChunk, n - c0);
+    float m = -INFINITY;
+    for (int s = threadIdx.x; s < cn; s += kMergeThreads)
+      m = fmaxf(m, __ldg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h));
+    const float M_new = fmaxf(M, block_max(m, red));
+    if (M_new == -INFINITY) continue;  // nothing finite so far
+    const float r = expf(M - M_new);   // 0 while M is -inf
+    float part = 0.f;
+    for (int s = threadIdx.x; s < cn; s += kMergeThreads) {
+      const float w = expf(__ldg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h) - M_new);
+      wsh[s] = w;
+      part += w;
     }
-    o /= l;
+    L = L * r + block_sum(part, red);  // block_sum's barriers also publish wsh
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[j] *= r;
+    for (int s = warp; s < cn; s += kMergeWarps) {
+      const float w = wsh[s];
+      const float* row = p.o_part + ((size_t)(base + c0 + s) * p.Hq + h) * D + P * lane;
+      if constexpr (P == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(row));
+        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
+      } else {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(row));
+        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
+      }
+    }
+    M = M_new;
+    __syncthreads();  // wsh is rewritten by the next chunk
   }
-  p.o[((size_t)b * p.Hq + h) * D + i] = o;
-  if (i == 0) p.lse[(size_t)b * p.Hq + h] = (m == -INFINITY) ? -INFINITY : m + logf(l);
+#pragma unroll
+  for (int j = 0; j < P; ++j) acc_sh[warp][P * lane + j] = acc[j];
+  __syncthreads();
+  for (int i = threadIdx.x; i < D; i += kMergeThreads) {
+    float o = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kMergeWarps; ++w) o += acc_sh[w][i];
+      o /= L;
+    }
+    p.o[((size_t)b * p.Hq + h) * D + i] = o;
+  }
+  if (threadIdx.x == 0) p.lse[(size_t)b * p.Hq + h] = (M == -INFINITY) ? -INFINITY : M + logf(L);
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s) {
   dim3 grid(p.n_seq, p.Hq);
-  if (d == 128) merge_kernel<128><<<grid, 128, 0, s>>>(p);
-  else merge_kernel<64><<<grid, 64, 0, s>>>(p);
+  if (d == 128) merge_kernel<128><<<grid, kMergeThreads, 0, s>>>(p);
+  else merge_kernel<64><<<grid, kMergeThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
