@@ -39,7 +39,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny"])
+    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny", "staged"])
+    ap.add_argument("--layers", type=int, default=None, help="staged workload: layers (default 16)")
     ap.add_argument("--variant", default="auto", choices=["auto", "simt", "mma"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.5,
@@ -148,6 +149,9 @@ def describe(name, wl, w):
         "tiny": "tiny exact decode: batch 1, 1 q / 1 KV head, d 64, 256 BF16 tokens, 4 splits of 64",
         "hybrid": "hybrid tier: batch 4, 32 q / 8 KV heads, d 128, 32768 tokens (newest 2048 BF16, 30720 4-bit codes)",
         "ragged": "ragged paged hybrid: batch 64, lengths U[1024, 65536], 16-token pages, newest 1024 BF16",
+        "staged": "staged 128k history: batch 1, 16 layers, 32 q / 8 KV heads, d 128, 131072 BF16 tokens per layer "
+                  "in pinned host memory, 4096-token chunks through a 2-buffer device region, one token appended "
+                  "per step",
     }[name], "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.d, "split_tokens": wl.split_tokens,
         "kv_bytes_per_step": w.kv_bytes()}
     d["l2"] = ("inputs larger than the 126 MB L2, no flush" if w.kv_bytes() > 126e6
@@ -191,6 +195,17 @@ def oracle_sequence_fn(name, wl, seed_rank=0):
             ora.decode_sequence(f64(q[b, h * G:(h + 1) * G]), tiers, wl.scale, wl.split_tokens)
             return T / wl.Hkv
         return fn, wl.B * wl.Hkv, "one (sequence, KV head) with its 4 query heads per unit, encode included"
+    if name == "staged":
+        n = 16384  # tokens of one layer per unit (a bounded sample of the 131072-token layer)
+        gen = synth.stream(wl.seed, "oracle-sample")
+
+        def fn(i):
+            k = synth.normal_bf16(gen, (wl.Hkv, n, wl.d))
+            v = synth.normal_bf16(gen, (wl.Hkv, n, wl.d))
+            q = synth.normal_bf16(gen, (wl.Hq, wl.d))
+            ora.decode_sequence(f64(q), [(f64(k), f64(v))], wl.scale, wl.split_tokens)
+            return n
+        return fn, 4, "one layer's decode over a 16384-token sample of its history per unit"
     lens = synth.ragged_lengths(wl)
     q = synth.queries(wl)
 
@@ -404,10 +419,98 @@ def run_ours(args):
     return 0
 
 
+def run_staged(args):
+    """Staged 128k decode: PCIe-bound, timed by host wall clock around an uninstrumented loop
+    (timing-enabled events serialise the copies they observe); one replica per rank."""
+    import torch
+    from kv_cache_tiering_b200 import akv, synth, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    base = synth.WORKLOADS["staged"]
+    wl = synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.d, base.split_tokens, seed=base.seed + rank,
+                        extra=dict(base.extra))
+    layers = args.layers or wl.extra["layers"]
+    n_steps = max(3, args.warmup) + args.steps
+    st = workloads.StagedDecode(wl, dev, layers=layers, max_steps=n_steps + 1)
+    variant = {"auto": akv.AKV_VARIANT_AUTO, "simt": akv.AKV_VARIANT_SIMT, "mma": akv.AKV_VARIANT_MMA}[args.variant]
+    inputs = [st.inputs(i) for i in range(n_steps)]
+    # pinned host -> device copy bandwidth of this box (the PCIe roofline)
+    probe_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    probe_d = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        probe_d.copy_(probe_h, non_blocking=True)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(5):
+        probe_d.copy_(probe_h, non_blocking=True)
+    torch.cuda.synchronize()
+    pcie_peak = 5 * probe_h.numel() / (time.perf_counter() - t0) / 1e9
+    del probe_h, probe_d
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(max(3, args.warmup)):
+        st.step(*inputs[i], variant)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    h2d0 = st.h2d_bytes
+    tw0 = time.monotonic()
+    t0 = time.perf_counter()
+    for i in range(max(3, args.warmup), n_steps):
+        st.step(*inputs[i], variant)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    tw1 = time.monotonic()
+    if dist:
+        t = torch.tensor([dt], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dt = float(t.item())
+    sampler.stop()
+    h2d = st.h2d_bytes - h2d0
+    n_tok = sum(layers * (wl.extra["T"] + i + 1) for i in range(max(3, args.warmup), n_steps))
+    value = n_tok * world / dt
+    err = int(st.err.item())
+    st.close()
+    if rank == 0:
+        pcie = h2d / dt / 1e9
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "staged 128k history: batch 1, %d layers, 32 q / 8 KV heads, d 128, "
+                                       "131072 BF16 tokens per layer in pinned host memory, 4096-token chunks "
+                                       "through a 2-buffer device region, one token appended per step" % layers,
+                           "timing": "host wall clock, timing-disabled fences", "parallelism":
+                           f"independent replicas x{world}", "variant": args.variant},
+                "roofline": {"bound": "pcie", "achieved": pcie, "peak": pcie_peak, "unit": "GB/s",
+                             "frac": pcie / pcie_peak, "traffic": None,
+                             "peak_source": "pinned 256 MiB host-to-device copy measured in this run"},
+                "pcie_h2d_gbs": pcie, "h2d_bytes_per_step": h2d // args.steps,
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d // args.steps,
+                        "d2h_bytes_per_step": layers * st.row_bytes},
+                "gpu_launches": args.steps * layers * (-(-(wl.extra["T"] + 1) // st.chunk) + 1),
+                "clocks": sampler.summary(tw0, tw1), "device_error_word": err}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "staged":
+        return run_staged(args)
     return run_ours(args)
 
 

@@ -213,7 +213,8 @@ akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, i
  * akv_stage_chunk: take the next buffer; make sure every event on its list has fired;
  *   copy `bytes` from pinned_src (page-locked host memory, else AKV_ERR_NOT_PINNED) with
  *   cudaMemcpyAsync on copy_stream; record the copy's event.  bytes larger than one
- *   buffer gives AKV_ERR_BUDGET.  timeout_ms >= 0: the host polls the events for at most
+ *   buffer gives AKV_ERR_BUDGET; bytes == 0 acquires the buffer without copying (the
+ *   caller fills it on the device).  timeout_ms >= 0: the host polls the events for at most
  *   timeout_ms and returns AKV_ERR_TIMEOUT, leaving the buffer untouched, if one is still
  *   pending.  timeout_ms < 0: the host does not wait; copy_stream waits for the events
  *   on the device instead.  Returns the buffer index and its device address.

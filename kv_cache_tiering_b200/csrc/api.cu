@@ -439,11 +439,10 @@ akv_status akv_stager_create(void* dev_region, size_t region_bytes, int n_buffer
 
 akv_status akv_stage_chunk(akv_stager* st, const void* pinned_src, size_t bytes, akv_stream_t copy_stream,
                            int timeout_ms, int* buf_index, void** dev_ptr) {
-  if (!st || !pinned_src || !buf_index || !dev_ptr) return fail(AKV_ERR_INVALID, "null argument");
-  if (bytes == 0) return fail(AKV_ERR_INVALID, "empty chunk");
+  if (!st || (!pinned_src && bytes) || !buf_index || !dev_ptr) return fail(AKV_ERR_INVALID, "null argument");
   if (bytes > st->buf_bytes)
     return fail(AKV_ERR_BUDGET, "chunk of %zu bytes exceeds the %zu-byte staging buffer", bytes, st->buf_bytes);
-  if (!is_pinned(pinned_src) || !is_pinned(static_cast<const uint8_t*>(pinned_src) + bytes - 1))
+  if (bytes && (!is_pinned(pinned_src) || !is_pinned(static_cast<const uint8_t*>(pinned_src) + bytes - 1)))
     return fail(AKV_ERR_NOT_PINNED, "staging source is not page-locked host memory");
   const int idx = st->next;
   akv_stager::Buffer& buf = st->bufs[idx];
@@ -473,8 +472,9 @@ akv_status akv_stage_chunk(akv_stager* st, const void* pinned_src, size_t bytes,
   buf.pending.clear();
   buf.ready = nullptr;
   uint8_t* dst = st->region + (size_t)idx * st->buf_bytes;
-  cudaError_t e = cudaMemcpyAsync(dst, pinned_src, bytes, cudaMemcpyHostToDevice, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync H2D");
+  cudaError_t e = cudaSuccess;
+  if (bytes && (e = cudaMemcpyAsync(dst, pinned_src, bytes, cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyAsync H2D");
   cudaEvent_t ev;
   if ((e = take_event(st, &ev)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
   if ((e = cudaEventRecord(ev, cs)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");

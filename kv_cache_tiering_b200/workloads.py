@@ -193,3 +193,112 @@ class RaggedPaged:
     def kv_bytes(self) -> int:
         d, H = self.wl.d, self.wl.Hkv
         return int(H * (2 * self.ex_len.sum() * d * 2 + 2 * self.cp_len.sum() * (d // 2 + 2)))
+
+
+class StagedDecode:
+    """Host-authoritative history staged through a bounded device ring.
+
+    Each layer's history lives in pinned host memory as rows [token][K|V][Hkv][d], so any
+    run of tokens is one contiguous span.  A decode step, per layer: every 4096-token chunk
+    is copied into the next ring buffer (akv_stage_chunk on the copy stream), the new
+    token's K/V is appended into the chunk that holds its position, the chunk's splits are
+    attended on the compute stream, the new row is written back to the host copy, and the
+    buffer is released; the layer's split partials are then merged.  ``resident=True``
+    keeps the same chunks in device memory instead and issues the same attend calls, which
+    is the comparison run for bit-identity."""
+
+    def __init__(self, wl: synth.Workload, device, layers: int | None = None, T: int | None = None,
+                 chunk: int | None = None, max_steps: int = 8, n_buffers: int = 2, resident: bool = False,
+                 host_layers=None):
+        self.wl, self.device, self.resident = wl, device, resident
+        self.L = wl.extra["layers"] if layers is None else layers
+        self.T = wl.extra["T"] if T is None else T
+        self.chunk = wl.extra["chunk"] if chunk is None else chunk
+        H, d = wl.Hkv, wl.d
+        self.row_elems = 2 * H * d
+        self.row_bytes = 2 * self.row_elems
+        cap = self.T + max_steps
+        self.cap = -(-cap // self.chunk) * self.chunk
+        if host_layers is None:
+            host_layers = []
+            for layer in range(self.L):
+                k, v = synth.history_token_major(wl, layer, self.T)
+                h = torch.empty((self.cap, 2, H, d), dtype=torch.int16).pin_memory()
+                h[: self.T, 0] = torch.from_numpy(k.view(np.int16))
+                h[: self.T, 1] = torch.from_numpy(v.view(np.int16))
+                host_layers.append(h)
+        self.host = host_layers
+        self.copy_stream = torch.cuda.Stream(device)
+        self.compute_stream = torch.cuda.Stream(device)
+        if resident:
+            self.dev_layers = [h.to(device) for h in self.host]
+        else:
+            self.region = torch.empty(n_buffers * self.chunk * self.row_bytes, dtype=torch.uint8, device=device)
+            self.stager = akv.Stager(self.region, self.region.numel(), n_buffers)
+        n_slots = -(-self.cap // wl.split_tokens)
+        self.o_part = torch.empty((n_slots, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty((n_slots, wl.Hq), dtype=torch.float32, device=device)
+        self.o = torch.empty((self.L, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse = torch.empty((self.L, wl.Hq), dtype=torch.float32, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.steps_done = 0
+        self.h2d_bytes = 0
+
+    def inputs(self, step: int):
+        """Device q [L][Hq][d] and new rows [L][2][Hkv][d] of decode step ``step``."""
+        q = np.stack([synth.queries(self.wl, layer=l, step=step, B=1)[0] for l in range(self.L)])
+        new = np.stack([np.stack(synth.new_token(self.wl, l, step)) for l in range(self.L)])
+        return to_dev_bits(q, self.device), to_dev_bits(new, self.device)
+
+    def step(self, q, new_rows, variant=akv.AKV_VARIANT_AUTO, timeout_ms: int = -1):
+        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device)."""
+        wl, H, d = self.wl, self.wl.Hkv, self.wl.d
+        pos = self.T + self.steps_done          # position of the appended token
+        n_tok = pos + 1
+        cs = self.compute_stream
+        n_chunks = -(-n_tok // self.chunk)
+        n_split = -(-n_tok // wl.split_tokens)
+        per_chunk = self.chunk // wl.split_tokens
+        rb = self.row_bytes
+        for layer in range(self.L):
+            new_row = new_rows[layer].reshape(-1).view(torch.uint8)
+            for c in range(n_chunks):
+                tok0 = c * self.chunk
+                ntc = min(self.chunk, n_tok - tok0)
+                have = min(self.chunk, pos - tok0)  # rows already in the host copy
+                appends = tok0 <= pos < tok0 + self.chunk
+                buf = None
+                if self.resident:
+                    store = self.dev_layers[layer].view(torch.uint8).reshape(-1)
+                    off = tok0 * rb
+                else:
+                    src = self.host[layer].data_ptr() + tok0 * rb
+                    buf, dev = self.stager.stage_chunk(src, have * rb, self.copy_stream, timeout_ms)
+                    self.h2d_bytes += have * rb
+                    self.stager.use(buf, cs)
+                    store = self.region
+                    off = dev - self.region.data_ptr()
+                base = store.data_ptr() + off
+                with torch.cuda.stream(cs):
+                    if appends:  # the new token's row goes into the chunk that holds its position
+                        store[off + (pos - tok0) * rb: off + (pos - tok0 + 1) * rb].copy_(new_row)
+                    tier = akv.Tier(akv.AKV_TIER_BF16, base, base + H * d * 2, lens=[ntc],
+                                    slot_base=[c * per_chunk], stride_seq=0, stride_head=d, stride_token=2 * H * d)
+                    akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
+                                          self.lse_part, self.o_part.shape[0], variant, self.err, cs)
+                    if appends:  # write the new row back to the authoritative host copy
+                        if self.resident:
+                            self.host[layer][pos].view(torch.uint8).reshape(-1).copy_(
+                                store[off + (pos - tok0) * rb: off + (pos - tok0 + 1) * rb], non_blocking=True)
+                        else:
+                            self.stager.writeback(buf, (pos - tok0) * rb, self.host[layer].data_ptr() + pos * rb,
+                                                  rb, cs)
+                if buf is not None:
+                    self.stager.release(buf, cs)
+            akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [n_split], 1, wl.Hq, d,
+                              self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
+        self.steps_done += 1
+
+    def close(self):
+        if not self.resident:
+            self.stager.destroy()
