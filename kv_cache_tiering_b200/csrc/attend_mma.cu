@@ -610,9 +610,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   }
   __syncthreads();
 
-  // this warp's item range: an equal share of all items, in item order
+  // this warp's item range: an equal share of all items, in item order; warps are numbered
+  // warp-major across CTAs so a partly filled grid still spreads its busy warps over every SM
   const int total = p.seq.item_base[p.seq.n_seq];
-  const int nw = (int)gridDim.x * NWARP, gw = (int)blockIdx.x * NWARP + warp;
+  const int nw = (int)gridDim.x * NWARP, gw = warp * (int)gridDim.x + (int)blockIdx.x;
   const int q0 = total / nw, r0 = total % nw;
   const int lo = gw * q0 + min(gw, r0), hi = lo + q0 + (gw < r0 ? 1 : 0);
   if (lo >= hi) return;
@@ -916,8 +917,7 @@ cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
-  const int want = (n_items + NWARP - 1) / NWARP;
-  const int grid = want < sms ? want : sms;
+  const int grid = n_items < sms ? n_items : sms;
   k<<<grid, NWARP * 32, C::SMEM, s>>>(p);
   return cudaGetLastError();
 }

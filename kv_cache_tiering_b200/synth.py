@@ -151,3 +151,33 @@ def scatter_pages(tokens_hd: np.ndarray, table_row: np.ndarray, pool: np.ndarray
     for j in range(n_pages):
         a, e = j * PAGE_TOKENS, min((j + 1) * PAGE_TOKENS, T)
         pool[table_row[j], :, : e - a, :] = tokens_hd[:, a:e, :]
+
+
+# ----------------------------------------------------------------------------------
+# device-side generators for full-size workloads (same distributions, BF16 rounding RNE)
+# ----------------------------------------------------------------------------------
+
+
+def torch_generator(seed: int, *key, device="cuda"):
+    """A seeded torch generator on `device` for (seed, key...)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(stream(seed, "torch", *key).integers(0, 2**62)))
+    return g
+
+
+def torch_normal_bf16(g, shape, device="cuda"):
+    """N(0,1) rounded to BF16; returns an int16 tensor holding the BF16 bits."""
+    import torch
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return x.to(torch.bfloat16).view(torch.int16)
+
+
+def torch_student_t3_bf16(g, shape, device="cuda"):
+    """Student-t with 3 degrees of freedom, z / sqrt((z1^2 + z2^2 + z3^2) / 3), rounded to BF16."""
+    import torch
+    z = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    chi2 = torch.zeros(shape, device=device, dtype=torch.float32)
+    for _ in range(3):
+        chi2.add_(torch.randn(shape, generator=g, device=device, dtype=torch.float32).square_())
+    return (z / torch.sqrt(chi2 / 3.0)).to(torch.bfloat16).view(torch.int16)

@@ -135,7 +135,7 @@ class RaggedPaged:
     [P, Hkv, 16, d]), the rest compact (code-block pool [P, Hkv])."""
 
     def __init__(self, wl: synth.Workload, device, B: int | None = None, lens=None, W: int | None = None,
-                 key_dist: str = "student_t"):
+                 key_dist: str = "student_t", generator: str = "numpy"):
         self.wl = wl
         B = wl.B if B is None else B
         W = wl.extra["window"] if W is None else W
@@ -166,6 +166,13 @@ class RaggedPaged:
                                    page_table=self.ex_table, page_table_stride=self.ex_table_np.shape[1],
                                    n_pages=n_ex, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
         self.key_dist = key_dist
+        self.ex_len, self.cp_len = ex_len, cp_len
+        self.step = None
+        if generator == "torch":
+            self._fill_on_device(wl, device, lens, ex_len, cp_len, n_cp)
+            self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [self.codes_tier, self.exact_tier],
+                                   device)
+            return
         ex_pool_k = np.zeros((n_ex, H, 16, d), np.uint16)
         ex_pool_v = np.zeros((n_ex, H, 16, d), np.uint16)
         for b in range(B):
@@ -189,6 +196,33 @@ class RaggedPaged:
         self.ex_v.copy_(torch.from_numpy(ex_pool_v.view(np.int16)))
         self.ex_len, self.cp_len = ex_len, cp_len
         self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [self.codes_tier, self.exact_tier], device)
+
+    def _fill_on_device(self, wl, device, lens, ex_len, cp_len, n_cp):
+        """Full-size fill: draw each sequence on the device (seeded torch generators), encode
+        its compact part through the library and scatter its exact part into the page pool."""
+        d, H = wl.d, wl.Hkv
+        for b in range(self.B):
+            L, c = int(lens[b]), int(cp_len[b])
+            g = synth.torch_generator(wl.seed, wl.name, "kv", b, device=device)
+            k = synth.torch_student_t3_bf16(g, (H, L, d), device) if self.key_dist == "student_t" \
+                else synth.torch_normal_bf16(g, (H, L, d), device)
+            v = synth.torch_normal_bf16(g, (H, L, d), device)
+            if c > 0:
+                src = akv.Tier(akv.AKV_TIER_BF16, k, v, lens=[c], stride_seq=0, stride_head=L * d, stride_token=d)
+                dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True,
+                               page_table=self.cp_table[b:b + 1], page_table_stride=self.cp_table_np.shape[1],
+                               n_pages=n_cp, stride_seq=H, stride_head=1)
+                akv.akv_encode_history(src, dst, 1, H, d, self.enc_err)
+            e = int(ex_len[b])
+            pages = -(-e // 16)
+            ex_k = torch.zeros((H, pages * 16, d), dtype=torch.int16, device=device)
+            ex_v = torch.zeros((H, pages * 16, d), dtype=torch.int16, device=device)
+            ex_k[:, :e] = k[:, c:]
+            ex_v[:, :e] = v[:, c:]
+            rows = self.ex_table[b, :pages].long()
+            self.ex_k[rows] = ex_k.view(H, pages, 16, d).permute(1, 0, 2, 3)
+            self.ex_v[rows] = ex_v.view(H, pages, 16, d).permute(1, 0, 2, 3)
+        torch.cuda.synchronize(device)
 
     def kv_bytes(self) -> int:
         d, H = self.wl.d, self.wl.Hkv
