@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--soak-seconds", type=float, default=1.5,
                     help="untimed steady-state run before the timed region (clocks settle, samples taken)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fuse", action="store_true",
+                    help="the fused decode call (merge folded into the attention launches) instead of separate "
+                         "attention and merge launches")
     return ap.parse_args()
 
 
@@ -138,7 +141,7 @@ def make_workload(name: str, device, rank: int):
         w = workloads.HybridResident(wl, device)
         tokens = w.B * w.T
     else:
-        w = workloads.RaggedPaged(wl, device)
+        w = workloads.RaggedPaged(wl, device, generator="torch")
         tokens = int(w.lens.sum())
     return wl, w, tokens
 
@@ -302,12 +305,21 @@ def run_ours(args):
     if w.kv_bytes() <= 126e6:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    fuse = args.fuse and variant != akv.AKV_VARIANT_SIMT
+
+    def run_step(q):
+        if fuse:
+            step.decode(q, variant, stream)
+        else:
+            step.step(q, variant, stream)
+
     def one_step():
         if flush is not None:
             flush.fill_(1)
-        step.step(w.q, variant, stream)
+        run_step(w.q)
 
-    launches_per_step = sum(1 for t in step.tiers if int(sum(t.lens)) > 0) + 1  # attends + merge (B <= 256)
+    # attention launches (one per non-empty tier, B <= 256), plus the merge unless fused
+    launches_per_step = sum(1 for t in step.tiers if int(sum(t.lens)) > 0) + (0 if fuse else 1)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -334,9 +346,13 @@ def run_ours(args):
         if flush is not None:
             flush.fill_(1)
         a0[i].record(stream)
-        step.attend(w.q, variant, stream)
+        if fuse:
+            step.decode(w.q, variant, stream)
+        else:
+            step.attend(w.q, variant, stream)
         a1[i].record(stream)
-        step.merge(stream)
+        if not fuse:
+            step.merge(stream)
     end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.monotonic()
@@ -373,7 +389,7 @@ def run_ours(args):
         q_dev.copy_(q_host, non_blocking=True)
         if flush is not None:
             flush.fill_(1)
-        step.step(q_dev, variant, stream)
+        run_step(q_dev)
         o_host.copy_(step.o, non_blocking=True)
         lse_host.copy_(step.lse, non_blocking=True)
     e1.record(stream)
@@ -398,10 +414,13 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(describe(args.workload, wl, w), parallelism=f"independent replicas x{world}",
-                               accumulate="f32", variant=args.variant),
+                               accumulate="f32", variant=args.variant,
+                               step="fused decode call (attention + merge)" if fuse
+                               else "attention launches + merge launch"),
                 "hbm_gbs": kv_bytes * world * args.steps / (ms * 1e-3) / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": None, "kernel": "akv attend (all tiers of a step)",
+                             "frac": achieved / peak, "traffic": None,
+                             "kernel": "akv attention launches of a step" + (" (merge fused in)" if fuse else ""),
                              "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
                              "attend_ms_avg": attend_avg_ms},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(q_host.numel() * 2),

@@ -190,6 +190,30 @@ akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_s
                          int d, float* o, float* lse, akv_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * akv_decode -- one whole decode step in one call: the split attention of every tier and
+ * the exact log-sum-exp merge ("Context beyond VRAM", "What I built": recent context
+ * exact, older history compact, the two merged with exact attention arithmetic).
+ *
+ * The result equals akv_decode_attend followed by akv_merge_lse with the akv_plan_slots
+ * layout (up to float32 rounding of the merge order), without a separate merge launch:
+ * every finished split bumps a per-(sequence, KV head) counter and the split that
+ * completes a sequence merges its query heads from the L2-resident partials.  Tiers'
+ * slot_base arrays are ignored (the call plans its own slots).
+ *
+ * workspace: caller-owned device scratch of at least akv_decode_workspace_size() bytes,
+ * 256-byte aligned, holding the counters, then the LSE and O partials.  Zero it once after
+ * allocating it; every call leaves the counters at zero again.  Calls that share a
+ * workspace must not overlap on the device.  o, lse: device float32 [B][Hq][d], [B][Hq].
+ * A smaller workspace gives AKV_ERR_BUDGET.  variant AKV_VARIANT_SIMT runs the CUDA-core
+ * attention and the separate merge.
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_decode_workspace_size(int B, int Hq, int Hkv, int d, const akv_tier* tiers, int n_tiers,
+                                     int split_tokens, size_t* bytes);
+akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
+                      int n_tiers, int split_tokens, void* workspace, size_t workspace_bytes, float* o, float* lse,
+                      int variant, int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * akv_plan_slots -- host helper: the standard slot layout.
  *
  * Sequence-major: sequence b owns a contiguous run of slots holding tier 0's splits,

@@ -29,6 +29,7 @@ AKV_ERR_BOUNDS = -9
 AKV_EFLAG_NONFINITE = 0x1
 AKV_EFLAG_RANGE = 0x2
 AKV_EFLAG_BOUNDS = 0x4
+AKV_EFLAG_TIMEOUT = 0x8
 
 AKV_TIER_BF16 = 0
 AKV_TIER_CODES4 = 1
@@ -97,6 +98,10 @@ _sig("akv_decode_attend", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, _p, ctypes.c_int64, ctypes.c_int, _p, _p)
 _sig("akv_merge_lse", ctypes.c_int, _p, _p, ctypes.c_int64, _p, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p, _p,
      _p)
+_sig("akv_decode_workspace_size", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t))
+_sig("akv_decode", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, _p, _p)
 _sig("akv_stager_create", ctypes.c_int, _p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_p))
 _sig("akv_stage_chunk", ctypes.c_int, _p, _p, ctypes.c_size_t, _p, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
      ctypes.POINTER(_p))
@@ -107,7 +112,8 @@ _sig("akv_stager_destroy", ctypes.c_int, _p)
 
 EXPORTED = [
     "akv_abi_version", "akv_last_error", "akv_status_string", "akv_error_word_status", "akv_centroids_f16",
-    "akv_plan_slots", "akv_encode_history", "akv_decode_attend", "akv_merge_lse", "akv_stager_create",
+    "akv_plan_slots", "akv_encode_history", "akv_decode_attend", "akv_merge_lse", "akv_decode_workspace_size",
+    "akv_decode", "akv_stager_create",
     "akv_stage_chunk", "akv_stager_use", "akv_stager_release", "akv_stage_writeback", "akv_stager_destroy",
 ]
 
@@ -229,6 +235,23 @@ def akv_merge_lse(o_part, lse_part, n_slots: int, seq_slot_base, seq_n_slots, B:
     cnt = _host_i32(seq_n_slots)
     _check(lib.akv_merge_lse(_ptr(o_part), _ptr(lse_part), int(n_slots), base.ctypes.data, cnt.ctypes.data, B, Hq,
                              d, _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def akv_decode_workspace_size(B: int, Hq: int, Hkv: int, d: int, tiers, split_tokens: int) -> int:
+    cs = [t.c() for t in tiers]
+    arr = (AkvTierC * max(1, len(cs)))(*cs)
+    n = ctypes.c_size_t(0)
+    _check(lib.akv_decode_workspace_size(B, Hq, Hkv, d, arr, len(cs), split_tokens, ctypes.byref(n)))
+    return n.value
+
+
+def akv_decode(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int, workspace,
+               workspace_bytes: int, o, lse, variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
+    cs = [t.c() for t in tiers]
+    arr = (AkvTierC * max(1, len(cs)))(*cs)
+    _check(lib.akv_decode(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens, _ptr(workspace),
+                          int(workspace_bytes), _ptr(o), _ptr(lse), variant, _ptr(err_word), _stream(stream)))
+    del cs
 
 
 class Stager:

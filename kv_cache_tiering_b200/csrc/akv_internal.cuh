@@ -37,6 +37,9 @@ struct SeqTable {
   int32_t item_base[kMaxSeqPerLaunch + 1];
   int32_t len[kMaxSeqPerLaunch];
   int32_t slot_base[kMaxSeqPerLaunch];
+  // fused decode: the sequence's slots over all tiers (merged by the item that completes them)
+  int32_t seq_slot_base[kMaxSeqPerLaunch];
+  int32_t seq_n_slots[kMaxSeqPerLaunch];
 };
 
 struct AttendParams {
@@ -50,6 +53,11 @@ struct AttendParams {
   int32_t Hq, Hkv, split_tokens;
   float scale_log2;      // softmax_scale * log2(e): scores are kept in base-2 units
   uint16_t centroids[16];
+  // fused decode: the item that completes a (sequence, KV head) also merges it into o / lse
+  int32_t fused;
+  int32_t* counters;     // [B][Hkv] finished splits; every merge resets its counter to 0
+  float* o;              // [B][Hq][D]
+  float* lse;            // [B][Hq]
   SeqTable seq;
 };
 

@@ -102,7 +102,8 @@ akv::TierDev tier_dev(const akv_tier* t) {
 // Fill st for sequences [b0, b0 + n): sequence b owns ceil(len / unit) * mult work
 // items; returns the total.
 int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, const int32_t* slot_base,
-                       int unit, int mult = 1) {
+                       int unit, int mult = 1, const int32_t* seq_slot_base = nullptr,
+                       const int32_t* seq_n_slots = nullptr) {
   st.n_seq = n;
   st.b0 = b0;
   int64_t items = 0;
@@ -110,15 +111,44 @@ int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, co
     st.item_base[i] = (int32_t)items;
     st.len[i] = lens[b0 + i];
     st.slot_base[i] = slot_base ? slot_base[b0 + i] : 0;
+    st.seq_slot_base[i] = seq_slot_base ? seq_slot_base[b0 + i] : 0;
+    st.seq_n_slots[i] = seq_n_slots ? seq_n_slots[b0 + i] : 0;
     items += ceil_div(lens[b0 + i], unit) * mult;
   }
   st.item_base[n] = (int32_t)items;
   for (int i = n; i < akv::kMaxSeqPerLaunch; ++i) {
     st.len[i] = 0;
     st.slot_base[i] = 0;
+    st.seq_slot_base[i] = 0;
+    st.seq_n_slots[i] = 0;
     st.item_base[i + 1] = (int32_t)items;
   }
   return items;
+}
+
+// Fused decode: where the partials are merged.
+struct FusedArgs {
+  int32_t* counters;
+  float* o;
+  float* lse;
+  const int32_t* seq_slot_base;  // host [B]
+  const int32_t* seq_n_slots;    // host [B]
+};
+
+// Byte layout of a fused-decode workspace: counters [B][Hkv] int32, LSE partials
+// [n_slots][Hq] float, O partials [n_slots][Hq][d] float, each 256-byte aligned.
+struct WorkspaceLayout {
+  size_t counters, lse, o, total;
+};
+
+WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  WorkspaceLayout l;
+  l.counters = 0;
+  l.lse = up((size_t)B * Hkv * sizeof(int32_t));
+  l.o = l.lse + up((size_t)n_slots * Hq * sizeof(float));
+  l.total = l.o + up((size_t)n_slots * Hq * d * sizeof(float));
+  return l;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -268,9 +298,13 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
   return ok();
 }
 
-akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
-                             const akv_tier* tiers, int n_tiers, int split_tokens, float* o_part, float* lse_part,
-                             int64_t n_slots, int variant, int32_t* err_word, akv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
+                       int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
+                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused) {
   if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(AKV_ERR_INVALID, "Hq must be a positive multiple of Hkv");
   const int G = Hq / Hkv;
@@ -305,7 +339,10 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
   p.split_tokens = split_tokens;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   std::memcpy(p.centroids, akv::centroid_table_f16(), sizeof(p.centroids));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  p.fused = (fused && variant != AKV_VARIANT_SIMT) ? 1 : 0;
+  p.counters = fused ? fused->counters : nullptr;
+  p.o = fused ? fused->o : nullptr;
+  p.lse = fused ? fused->lse : nullptr;
   for (int i = 0; i < n_tiers; ++i) {
     p.tier = tier_dev(&tiers[i]);
     for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
@@ -314,7 +351,8 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
       // list of (split, KV head) items
       const bool simt = variant == AKV_VARIANT_SIMT;
       const int64_t items =
-          fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv);
+          fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv,
+                         fused ? fused->seq_slot_base : nullptr, fused ? fused->seq_n_slots : nullptr);
       if (items == 0) continue;
       if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
       if (!simt && tiers[i].kind == AKV_TIER_BF16) {
@@ -331,6 +369,17 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
     }
   }
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
+                             const akv_tier* tiers, int n_tiers, int split_tokens, float* o_part, float* lse_part,
+                             int64_t n_slots, int variant, int32_t* err_word, akv_stream_t stream) {
+  return attend_impl(q, B, Hq, Hkv, d, softmax_scale, tiers, n_tiers, split_tokens, o_part, lse_part, n_slots,
+                     variant, err_word, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_slots, const int32_t* seq_slot_base,
@@ -369,6 +418,72 @@ akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_s
     cudaError_t e = akv::launch_merge(p, d, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
+  return ok();
+}
+
+// Plan the standard slot layout for a fused decode (host vectors).
+static akv_status plan_for_decode(int B, const akv_tier* tiers, int n_tiers, int split_tokens,
+                                  std::vector<std::vector<int32_t>>& tier_base, std::vector<int32_t>& seq_base,
+                                  std::vector<int32_t>& seq_n, int64_t* n_slots) {
+  if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
+  if (n_tiers > 0 && !tiers) return fail(AKV_ERR_INVALID, "tiers is null");
+  if (split_tokens < 16 || split_tokens > akv::kMaxSplitTokens || split_tokens % 16)
+    return fail(AKV_ERR_UNSUPPORTED, "split_tokens %d (a multiple of 16 in [16, 1024])", split_tokens);
+  std::vector<const int32_t*> lens(n_tiers);
+  std::vector<int32_t*> bases(n_tiers);
+  tier_base.assign(n_tiers, std::vector<int32_t>(B > 0 ? B : 1));
+  for (int i = 0; i < n_tiers; ++i) {
+    if (!tiers[i].lens && B > 0) return fail(AKV_ERR_INVALID, "tier %d: lens is null", i);
+    lens[i] = tiers[i].lens;
+    bases[i] = tier_base[i].data();
+  }
+  seq_base.assign(B > 0 ? B : 1, 0);
+  seq_n.assign(B > 0 ? B : 1, 0);
+  return akv_plan_slots(B, n_tiers, lens.data(), split_tokens, bases.data(), seq_base.data(), seq_n.data(), n_slots);
+}
+
+akv_status akv_decode_workspace_size(int B, int Hq, int Hkv, int d, const akv_tier* tiers, int n_tiers,
+                                     int split_tokens, size_t* bytes) {
+  if (!bytes) return fail(AKV_ERR_INVALID, "bytes is null");
+  if (Hq <= 0 || Hkv <= 0 || d <= 0) return fail(AKV_ERR_INVALID, "Hq, Hkv and d must be positive");
+  std::vector<std::vector<int32_t>> tb;
+  std::vector<int32_t> sb, sn;
+  int64_t n_slots = 0;
+  akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
+  if (s != AKV_OK) return s;
+  *bytes = workspace_layout(B, Hq, Hkv, d, n_slots).total;
+  return ok();
+}
+
+akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
+                      int n_tiers, int split_tokens, void* workspace, size_t workspace_bytes, float* o, float* lse,
+                      int variant, int32_t* err_word, akv_stream_t stream) {
+  if (Hq <= 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "Hq and Hkv must be positive");
+  std::vector<std::vector<int32_t>> tb;
+  std::vector<int32_t> sb, sn;
+  int64_t n_slots = 0;
+  akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
+  if (s != AKV_OK) return s;
+  if (B == 0) return ok();
+  const WorkspaceLayout lay = workspace_layout(B, Hq, Hkv, d, n_slots);
+  if (!workspace || !aligned(workspace, 256)) return fail(AKV_ERR_INVALID, "workspace must be 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    return fail(AKV_ERR_BUDGET, "workspace of %zu bytes, %zu needed", workspace_bytes, lay.total);
+  if (!o || !lse) return fail(AKV_ERR_INVALID, "o and lse must not be null");
+  std::vector<akv_tier> planned(tiers, tiers + n_tiers);
+  for (int i = 0; i < n_tiers; ++i) planned[i].slot_base = tb[i].data();
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(ws + lay.lse);
+  float* o_part = reinterpret_cast<float*>(ws + lay.o);
+  FusedArgs fa{reinterpret_cast<int32_t*>(ws + lay.counters), o, lse, sb.data(), sn.data()};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = attend_impl(q, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
+                  n_slots, variant, err_word, st, &fa);
+  if (s != AKV_OK) return s;
+  // the CUDA-core path, and sequences without any token, take the separate merge
+  bool need_merge = variant == AKV_VARIANT_SIMT;
+  for (int b = 0; b < B && !need_merge; ++b) need_merge = sn[b] == 0;
+  if (need_merge) return akv_merge_lse(o_part, lse_part, n_slots, sb.data(), sn.data(), B, Hq, d, o, lse, stream);
   return ok();
 }
 

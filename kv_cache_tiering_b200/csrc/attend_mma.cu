@@ -136,6 +136,7 @@ __device__ __forceinline__ void group_sync(int gi) {
 // items
 // ------------------------------------------------------------------------------------
 struct Item {
+  int bl;     // sequence within the launch
   int b;      // global sequence
   int kvh;
   int t0;     // first token of the split (tier-relative)
@@ -153,6 +154,7 @@ __device__ __forceinline__ Item item_at(const AttendParams& p, int item) {
   Item it;
   it.kvh = r / ns;
   const int split = r - it.kvh * ns;
+  it.bl = bl;
   it.b = p.seq.b0 + bl;
   it.t0 = split * p.split_tokens;
   it.n = min(p.split_tokens, len - it.t0);
@@ -355,6 +357,41 @@ __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it
 }
 
 // ------------------------------------------------------------------------------------
+// fused decode: the item that completes a (sequence, KV head) merges its query heads
+// ------------------------------------------------------------------------------------
+// Every finished item fences its partial writes and bumps the (sequence, KV head) counter;
+// the item that brings it to the sequence's slot count merges slots seq_slot_base ..
+// + seq_n_slots - 1 in slot order (max, exp weights, weighted sum -- the LSE merge) and
+// resets the counter.  Partials of other CTAs are read past L1.
+template <int D, int G>
+__device__ __forceinline__ void merge_tail(const AttendParams& p, const Item& it, int t, int nthreads) {
+  const int base = p.seq.seq_slot_base[it.bl], n = p.seq.seq_n_slots[it.bl];
+  for (int i = t; i < G * D; i += nthreads) {
+    const int h = i / D, dim = i % D, hq = it.kvh * G + h;
+    float M = -INFINITY;
+    for (int s = 0; s < n; ++s) M = fmaxf(M, __ldcg(p.lse_part + (size_t)(base + s) * p.Hq + hq));
+    float o = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+      for (int s = 0; s < n; ++s) {
+        const float w = expf(__ldcg(p.lse_part + (size_t)(base + s) * p.Hq + hq) - M);
+        L += w;
+        o = fmaf(w, __ldcg(p.o_part + ((size_t)(base + s) * p.Hq + hq) * D + dim), o);
+      }
+      o /= L;
+    }
+    p.o[((size_t)it.b * p.Hq + hq) * D + dim] = o;
+    if (dim == 0) p.lse[(size_t)it.b * p.Hq + hq] = (M == -INFINITY) ? -INFINITY : M + logf(L);
+  }
+}
+
+// Count a finished item; true for the caller that completed the (sequence, KV head).
+__device__ __forceinline__ bool finish_item(const AttendParams& p, const Item& it) {
+  const int old = atomicAdd(p.counters + (size_t)it.b * p.Hkv + it.kvh, 1);
+  return old + 1 == p.seq.seq_n_slots[it.bl];
+}
+
+// ------------------------------------------------------------------------------------
 // exact BF16 tier
 // ------------------------------------------------------------------------------------
 template <int D, int G, int NW, int NST>
@@ -367,7 +404,8 @@ struct Bf16Cfg {
   static constexpr int AREA = NW * G * D;          // floats
   static constexpr int FLOATS = AREA + 3 * NW * G;  // area, m, l, factors
   static constexpr int BAR_OFF = RINGS + FLOATS * 4;
-  static constexpr size_t SMEM = BAR_OFF + NW * NST * 8 + 1024;  // + alignment slack
+  static constexpr int FLAG_OFF = BAR_OFF + NW * NST * 8;
+  static constexpr size_t SMEM = FLAG_OFF + 16 + 1024;  // + alignment slack
 };
 
 // Byte offset, inside a TMA-swizzled tile, of 16-byte chunk c (of D/8) of row r.
@@ -544,6 +582,18 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
     chain_to_smem<D, G>(acc, m_run, l_run, area + w * G * D, mws + w * G, lws + w * G, dim_of);
     group_sync<NW>(gi);
     merge_item<D, G, NW, false>(p, it, gi, area, mws, lws, fac, nullptr);
+    if (p.fused) {
+      int* flag = reinterpret_cast<int*>(smem + C::FLAG_OFF);
+      __threadfence();
+      group_sync<NW>(gi);
+      if (threadIdx.x == 0) *flag = finish_item(p, it) ? 1 : 0;
+      group_sync<NW>(gi);
+      if (*flag) {
+        __threadfence();
+        merge_tail<D, G>(p, it, threadIdx.x, NW * 32);
+        if (threadIdx.x == 0) p.counters[(size_t)it.b * p.Hkv + it.kvh] = 0;
+      }
+    }
     group_sync<NW>(gi);
   }
   if (!ok) {
@@ -880,6 +930,17 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
       } else {
         *reinterpret_cast<float2*>(dst) = make_float2(x[0], x[1]);
+      }
+    }
+    if (p.fused) {
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = finish_item(p, it) ? 1 : 0;
+      if (__shfl_sync(kFull, last, 0)) {
+        __threadfence();
+        merge_tail<D, G>(p, it, lane, 32);
+        if (lane == 0) p.counters[(size_t)it.b * p.Hkv + it.kvh] = 0;
       }
     }
     __syncwarp();

@@ -37,6 +37,13 @@ class DecodeStep:
         self.o = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
         self.lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws_bytes = akv.akv_decode_workspace_size(B, Hq, Hkv, d, tiers, split_tokens)
+        self.workspace = torch.zeros(max(256, self.ws_bytes), dtype=torch.uint8, device=device)
+
+    def decode(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        """The whole step in one call (split attention with the merge fused in)."""
+        akv.akv_decode(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens, self.workspace,
+                       self.ws_bytes, self.o, self.lse, variant, self.err, stream)
 
     def attend(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
         akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens,

@@ -361,3 +361,74 @@ def test_merge_special_values(akv, cuda):
             assert np.max(np.abs(o[b, h].cpu().numpy() - ro)) < 1e-5
             assert abs(lse[b, h].item() - rl) < 1e-5
     assert torch.all(o[2] == 0) and torch.all(lse[2] == -math.inf)
+
+
+# ----------------------------------------------------------------------------------
+# fused decode (attention with the merge folded in)
+# ----------------------------------------------------------------------------------
+
+
+def _fused_check(akv, step, q, refs_direct):
+    import torch
+    o_sep, l_sep = step.o.clone(), step.lse.clone()
+    step.o.fill_(float("nan"))
+    step.lse.fill_(float("nan"))
+    step.decode(q)
+    torch.cuda.synchronize()
+    counters = step.workspace[: 4 * step.B * step.Hkv].view(torch.int32)
+    assert int(counters.abs().sum().item()) == 0  # every counter is back at zero
+    assert float((step.o - o_sep).abs().max().item()) <= 1e-5
+    ls = step.lse.cpu().numpy().astype(np.float64)
+    lr = l_sep.cpu().numpy().astype(np.float64)
+    assert lse_diff(ls, lr) <= 1e-5
+    for b, ref in enumerate(refs_direct):
+        check_merged(step, b, ref)
+    o1, l1 = step.o.clone(), step.lse.clone()
+    step.decode(q)  # a second call on the same workspace gives the same bits
+    torch.cuda.synchronize()
+    assert torch.equal(o1, step.o) and torch.equal(l1, step.lse)
+
+
+def test_fused_decode_exact_full_size(akv, wlmod, cuda):
+    import torch
+    wl = synth.WORKLOADS["exact"]
+    w = wlmod.ExactResident(wl, cuda)
+    w.step.step(w.q)
+    torch.cuda.synchronize()
+    refs = [r[2] for r in _oracle_exact(wl, w.q_bits, w.k_bits, w.v_bits, [w.T] * w.B, wl.split_tokens)]
+    _fused_check(akv, w.step, w.q, refs)
+
+
+def test_fused_decode_ragged_paged_hybrid(akv, wlmod, cuda):
+    """Two launches (compact tier, then exact tier) share the counters; a sequence with
+    no compact tokens is completed by the exact launch."""
+    import torch
+    wl = synth.Workload("ragged-fused", B=5, Hq=32, Hkv=8, d=128, split_tokens=512,
+                        extra={"window": 1024, "nu": 3.0})
+    lens = np.array([700, 1024, 3000, 1500, 4100], np.int32)
+    w = wlmod.RaggedPaged(wl, cuda, lens=lens)
+    w.step.step(w.q)
+    torch.cuda.synchronize()
+    refs = []
+    for b in range(w.B):
+        k, v = synth.history_head_major(wl, b, int(lens[b]), key_dist="student_t")
+        c = int(w.cp_len[b])
+        kh = np.zeros((wl.Hkv, c, wl.d))
+        vh = np.zeros((wl.Hkv, c, wl.d))
+        for h in range(wl.Hkv):
+            if c:
+                ek, ev = ora.encode(k[h, :c]), ora.encode(v[h, :c])
+                kh[h] = ora.dequantize(ek.codes, ek.scale_bits)
+                vh[h] = ora.dequantize(ev.codes, ev.scale_bits)
+        tiers = [(kh, vh), (f64(k[:, c:]), f64(v[:, c:]))]
+        refs.append(ora.decode_sequence(f64(w.q_bits[b]), tiers, wl.scale, wl.split_tokens)[2])
+    _fused_check(akv, w.step, w.q, refs)
+
+
+def test_fused_decode_refuses_small_workspace(akv, wlmod, cuda):
+    wl = synth.WORKLOADS["tiny"]
+    w = wlmod.ExactResident(wl, cuda)
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_decode(w.q, w.B, wl.Hq, wl.Hkv, wl.d, wl.scale, w.step.tiers, wl.split_tokens, w.step.workspace,
+                       w.step.ws_bytes - 256, w.step.o, w.step.lse)
+    assert e.value.status == akv.AKV_ERR_BUDGET
