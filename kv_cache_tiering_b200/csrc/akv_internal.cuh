@@ -157,6 +157,30 @@ cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int
 cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int Hkv, int d, int64_t max_len);
 cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s);
 
+// Fused decode: where the partials are merged.
+struct FusedArgs {
+  int32_t* counters;
+  float* o;
+  float* lse;
+  const int32_t* seq_slot_base;  // host [B]
+  const int32_t* seq_n_slots;    // host [B]
+};
+
+// Byte layout of a fused-decode workspace: counters [B][Hkv] int32, LSE partials
+// [n_slots][Hq] float, O partials [n_slots][Hq][d] float, each 256-byte aligned.
+struct WorkspaceLayout {
+  size_t counters, lse, o, total;
+};
+WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots);
+
+// Validated split attention of every tier (fused != null: merge folded in).
+akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
+                       int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
+                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused);
+
+// Set the thread's last-error message; returns st.
+akv_status set_error(akv_status st, const char* msg);
+
 // host: the binary16 centroid table and its float64 decision boundaries
 const uint16_t* centroid_table_f16();
 const double* centroid_boundaries();

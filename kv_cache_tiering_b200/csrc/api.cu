@@ -126,20 +126,9 @@ int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, co
   return items;
 }
 
-// Fused decode: where the partials are merged.
-struct FusedArgs {
-  int32_t* counters;
-  float* o;
-  float* lse;
-  const int32_t* seq_slot_base;  // host [B]
-  const int32_t* seq_n_slots;    // host [B]
-};
+}  // namespace
 
-// Byte layout of a fused-decode workspace: counters [B][Hkv] int32, LSE partials
-// [n_slots][Hq] float, O partials [n_slots][Hq][d] float, each 256-byte aligned.
-struct WorkspaceLayout {
-  size_t counters, lse, o, total;
-};
+namespace akv {
 
 WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -165,9 +154,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-}  // namespace
 
-namespace akv {
 
 // TMA maps of a BF16 tier.  Logical outer coordinates: 0 token (in the page when paged),
 // 1 KV head, 2 sequence (page when paged).  The three outer dims are ordered by byte stride;
@@ -205,6 +192,8 @@ cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int
   }
   return cudaSuccess;
 }
+
+akv_status set_error(akv_status st, const char* msg) { return fail(st, "%s", msg); }
 
 }  // namespace akv
 
@@ -300,7 +289,7 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
 
 }  // extern "C"
 
-namespace {
+namespace akv {
 
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
@@ -371,14 +360,14 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
   return ok();
 }
 
-}  // namespace
+}  // namespace akv
 
 extern "C" {
 
 akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
                              const akv_tier* tiers, int n_tiers, int split_tokens, float* o_part, float* lse_part,
                              int64_t n_slots, int variant, int32_t* err_word, akv_stream_t stream) {
-  return attend_impl(q, B, Hq, Hkv, d, softmax_scale, tiers, n_tiers, split_tokens, o_part, lse_part, n_slots,
+  return akv::attend_impl(q, B, Hq, Hkv, d, softmax_scale, tiers, n_tiers, split_tokens, o_part, lse_part, n_slots,
                      variant, err_word, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
@@ -451,7 +440,7 @@ akv_status akv_decode_workspace_size(int B, int Hq, int Hkv, int d, const akv_ti
   int64_t n_slots = 0;
   akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
   if (s != AKV_OK) return s;
-  *bytes = workspace_layout(B, Hq, Hkv, d, n_slots).total;
+  *bytes = akv::workspace_layout(B, Hq, Hkv, d, n_slots).total;
   return ok();
 }
 
@@ -465,7 +454,7 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
   akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
   if (s != AKV_OK) return s;
   if (B == 0) return ok();
-  const WorkspaceLayout lay = workspace_layout(B, Hq, Hkv, d, n_slots);
+  const akv::WorkspaceLayout lay = akv::workspace_layout(B, Hq, Hkv, d, n_slots);
   if (!workspace || !aligned(workspace, 256)) return fail(AKV_ERR_INVALID, "workspace must be 256-byte aligned");
   if (workspace_bytes < lay.total)
     return fail(AKV_ERR_BUDGET, "workspace of %zu bytes, %zu needed", workspace_bytes, lay.total);
@@ -475,9 +464,9 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* lse_part = reinterpret_cast<float*>(ws + lay.lse);
   float* o_part = reinterpret_cast<float*>(ws + lay.o);
-  FusedArgs fa{reinterpret_cast<int32_t*>(ws + lay.counters), o, lse, sb.data(), sn.data()};
+  akv::FusedArgs fa{reinterpret_cast<int32_t*>(ws + lay.counters), o, lse, sb.data(), sn.data()};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  s = attend_impl(q, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
+  s = akv::attend_impl(q, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
                   n_slots, variant, err_word, st, &fa);
   if (s != AKV_OK) return s;
   // the CUDA-core path, and sequences without any token, take the separate merge
