@@ -214,6 +214,31 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
                       int variant, int32_t* err_word, akv_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * akv_decode_static -- akv_decode without a workspace argument, for callers that cannot
+ * allocate device memory when they decode (code inside a host function enqueued on a
+ * stream, where CUDA forbids calls such as cudaMalloc; a plugin whose process memory pool
+ * belongs to another framework; a serving loop that has frozen allocation so no call can
+ * block on the allocator or synchronise the device).  The pages have no counterpart:
+ * their engine always owns its memory.
+ *
+ * The scratch is a fixed array of AKV_DECODE_STATIC_MAX_BYTES in this library's device
+ * memory, held by every GPU that loads the library until the process exits; the call
+ * itself allocates nothing, on the device or the host.  A step whose partials do not fit
+ * (see akv_decode_workspace_size), or with more than AKV_DECODE_STATIC_MAX_SEQ sequences
+ * or 8 tiers, returns AKV_ERR_BUDGET / AKV_ERR_UNSUPPORTED and launches nothing.  The
+ * first call on each device looks up the array's device address while that device is
+ * current, so make it before any stream capture.  Every call shares the array: the
+ * completion counters are cleared at the start of each call, everything else keeps the
+ * last call's values, and calls whose work overlaps on the GPU race -- order them.
+ * Arguments and results are those of akv_decode.
+ * ------------------------------------------------------------------------------------ */
+#define AKV_DECODE_STATIC_MAX_BYTES (8u << 20)
+#define AKV_DECODE_STATIC_MAX_SEQ 1024
+akv_status akv_decode_static(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale,
+                             const akv_tier* tiers, int n_tiers, int split_tokens, float* o, float* lse,
+                             int variant, int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * akv_plan_slots -- host helper: the standard slot layout.
  *
  * Sequence-major: sequence b owns a contiguous run of slots holding tier 0's splits,

@@ -102,6 +102,8 @@ _sig("akv_decode_workspace_size", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctyp
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t))
 _sig("akv_decode", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, _p, _p)
+_sig("akv_decode_static", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, _p, ctypes.c_int, _p, _p)
 _sig("akv_stager_create", ctypes.c_int, _p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_p))
 _sig("akv_stage_chunk", ctypes.c_int, _p, _p, ctypes.c_size_t, _p, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
      ctypes.POINTER(_p))
@@ -251,6 +253,17 @@ def akv_decode(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers
     arr = (AkvTierC * max(1, len(cs)))(*cs)
     _check(lib.akv_decode(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens, _ptr(workspace),
                           int(workspace_bytes), _ptr(o), _ptr(lse), variant, _ptr(err_word), _stream(stream)))
+    del cs
+
+
+def akv_decode_static(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int, o, lse,
+                      variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
+    """akv_decode on the library's own fixed scratch, for callers that cannot allocate
+    device memory when they decode; see include/akv.h for its limits."""
+    cs = [t.c() for t in tiers]
+    arr = (AkvTierC * max(1, len(cs)))(*cs)
+    _check(lib.akv_decode_static(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens, _ptr(o),
+                                 _ptr(lse), variant, _ptr(err_word), _stream(stream)))
     del cs
 
 
