@@ -61,6 +61,30 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = ("kv_cache_tiering_b200/csrc/attend_mma.cu", "kv_cache_tiering_b200/csrc/akv_internal.cuh")
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload`, as one ncu capture
+    recorded them in profiles/dram_traffic.txt; None when nothing is recorded or the
+    kernel sources have changed since (their hash no longer matches the record)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    key = h.hexdigest()[:16]
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 5 and not line.startswith("#") and parts[:3] == [workload, kernel, key]:
+                return int(parts[3]) + int(parts[4])
+    return None
+
+
 # ----------------------------------------------------------------------------------
 # clocks sampled during the run
 # ----------------------------------------------------------------------------------
@@ -282,6 +306,14 @@ def run_reference(args):
 # ----------------------------------------------------------------------------------
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (every rank calls this, in the same order)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args):
     import torch
     from kv_cache_tiering_b200 import akv
@@ -333,9 +365,12 @@ def run_ours(args):
             one_step()
         torch.cuda.synchronize()
 
-    n_ev = args.steps
-    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    # events around every tier's launch, so the dominant kernel is timed on its own
+    live = [i for i, t in enumerate(step.tiers) if int(sum(t.lens)) > 0]
+    per_tier = not fuse and len(live) > 1
+    n_b = len(live) + 1 if per_tier else 2
+    bounds = [[torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] for _ in range(n_b)]
+    a0, a1 = bounds[0], bounds[-1]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -348,6 +383,10 @@ def run_ours(args):
         a0[i].record(stream)
         if fuse:
             step.decode(w.q, variant, stream)
+        elif per_tier:
+            for j, ti in enumerate(live):
+                step.attend_tier(ti, w.q, variant, stream)
+                bounds[j + 1][i].record(stream)
         else:
             step.attend(w.q, variant, stream)
         a1[i].record(stream)
@@ -360,10 +399,10 @@ def run_ours(args):
         dist.barrier()
     ms = start.elapsed_time(end)
     attend_ms = [a0[i].elapsed_time(a1[i]) for i in range(args.steps)]
+    tier_ms = ([statistics.fmean(bounds[j][i].elapsed_time(bounds[j + 1][i]) for i in range(args.steps))
+                for j in range(len(live))] if per_tier else None)
     if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dev)
     # post-timed soak so the sampler has points inside the loaded window
     t_post = time.monotonic()
     while time.monotonic() - t_post < 0.3:
@@ -396,9 +435,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     sampler.stop()
 
     total_tokens = tokens * world * args.steps
@@ -407,7 +444,22 @@ def run_ours(args):
     peak, peak_kind = peaks()
     attend_avg_ms = sum(attend_ms) / len(attend_ms)
     kv_bytes = w.kv_bytes()
-    achieved = kv_bytes / (attend_avg_ms * 1e-3) / 1e9
+    tb = w.tier_bytes()
+    kernel_names = ["attend_codes_mma" if step.tiers[i].kind == akv.AKV_TIER_CODES4 else "attend_bf16_mma"
+                    for i in live]
+    if variant == akv.AKV_VARIANT_SIMT:
+        kernel_names = [k.replace("_mma", "_simt") for k in kernel_names]
+    if per_tier:
+        # the dominant kernel: the tier launch with the largest share of the step
+        j = max(range(len(live)), key=lambda k: tier_ms[k])
+        dom_ms, dom_bytes, dom_kernel = tier_ms[j], tb[live[j]], kernel_names[j]
+    else:
+        dom_ms, dom_bytes = attend_avg_ms, kv_bytes
+        dom_kernel = kernel_names[0] if len(live) == 1 else "attention launches"
+        if fuse:
+            dom_kernel += " (merge fused in)"
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = None if fuse else recorded_traffic(args.workload, dom_kernel)
     clocks = sampler.summary(t_soak, t_wall1 + 0.3)
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -419,10 +471,11 @@ def run_ours(args):
                                else "attention launches + merge launch"),
                 "hbm_gbs": kv_bytes * world * args.steps / (ms * 1e-3) / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": None,
-                             "kernel": "akv attention launches of a step" + (" (merge fused in)" if fuse else ""),
+                             "frac": achieved / peak, "traffic": traffic, "kernel": dom_kernel,
+                             "algorithmic_bytes": dom_bytes, "kernel_ms_avg": dom_ms,
                              "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
-                             "attend_ms_avg": attend_avg_ms},
+                             "attend_ms_avg": attend_avg_ms,
+                             "tiers_ms_avg": dict(zip(kernel_names, tier_ms)) if per_tier else None},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(q_host.numel() * 2),
                         "d2h_bytes_per_step": int(o_host.numel() * 4 + lse_host.numel() * 4)},
                 "gpu_launches": launches_per_step * args.steps,

@@ -49,6 +49,11 @@ class DecodeStep:
         akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens,
                               self.o_part, self.lse_part, self.n_slots, variant, self.err, stream)
 
+    def attend_tier(self, i: int, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        """Tier i alone: the same launch ``attend`` makes for it, into the same slots."""
+        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, [self.tiers[i]], self.split_tokens,
+                              self.o_part, self.lse_part, self.n_slots, variant, self.err, stream)
+
     def merge(self, stream=None):
         akv.akv_merge_lse(self.o_part, self.lse_part, self.n_slots, self.seq_slot_base, self.seq_n_slots, self.B,
                           self.Hq, self.d, self.o, self.lse, stream)
@@ -91,6 +96,9 @@ class ExactResident:
     def kv_bytes(self) -> int:
         return 2 * self.B * self.wl.Hkv * self.T * self.wl.d * 2
 
+    def tier_bytes(self) -> list[int]:
+        return [self.kv_bytes()]
+
 
 class HybridResident:
     """Hybrid tiers of one batch: tokens [0, T - W) compact (contiguous code blocks
@@ -131,9 +139,13 @@ class HybridResident:
         self.step = DecodeStep(B, wl.Hq, H, d, wl.split_tokens, wl.scale, [self.codes_tier, exact], device)
 
     def kv_bytes(self) -> int:
+        return sum(self.tier_bytes())
+
+    def tier_bytes(self) -> list[int]:
+        """Bytes each tier's launch must read: K and V codes + fp16 norms, then BF16 K and V."""
         d, H = self.wl.d, self.wl.Hkv
         Tc = self.T - self.W
-        return self.B * H * (2 * self.W * d * 2 + 2 * Tc * (d // 2 + 2))
+        return [self.B * H * 2 * Tc * (d // 2 + 2), self.B * H * 2 * self.W * d * 2]
 
 
 class RaggedPaged:
@@ -232,8 +244,12 @@ class RaggedPaged:
         torch.cuda.synchronize(device)
 
     def kv_bytes(self) -> int:
+        return sum(self.tier_bytes())
+
+    def tier_bytes(self) -> list[int]:
+        """Bytes each tier's launch must read: compact pages' codes + norms, then BF16 pages."""
         d, H = self.wl.d, self.wl.Hkv
-        return int(H * (2 * self.ex_len.sum() * d * 2 + 2 * self.cp_len.sum() * (d // 2 + 2)))
+        return [int(H * 2 * self.cp_len.sum() * (d // 2 + 2)), int(H * 2 * self.ex_len.sum() * d * 2)]
 
 
 class StagedDecode:
