@@ -60,7 +60,9 @@ typedef enum akv_status {
   AKV_ERR_TIMEOUT = -6,      /* a staging buffer was still in use when the wait ran out */
   AKV_ERR_NONFINITE = -7,    /* device: an encoded vector held inf or NaN */
   AKV_ERR_RANGE = -8,        /* device: an encoded vector's norm overflows binary16 */
-  AKV_ERR_BOUNDS = -9        /* device: a page id outside [0, n_pages) */
+  AKV_ERR_BOUNDS = -9,       /* device: a page id outside [0, n_pages) */
+  AKV_ERR_INTERNAL = -10     /* device: a kernel got less shared memory than its layout needs
+                                (a library defect); it returned without reading or writing */
 } akv_status;
 
 /* Bits of the device error word. */
@@ -68,6 +70,7 @@ typedef enum akv_status {
 #define AKV_EFLAG_RANGE 0x2
 #define AKV_EFLAG_BOUNDS 0x4
 #define AKV_EFLAG_TIMEOUT 0x8 /* a kernel's bounded wait for its own copies gave up */
+#define AKV_EFLAG_INTERNAL 0x10 /* a kernel's shared-memory layout did not fit its launch */
 
 int akv_abi_version(void);
 const char* akv_last_error(void);
@@ -89,9 +92,16 @@ enum { AKV_TIER_BF16 = 0, AKV_TIER_CODES4 = 1 };
 /* Tokens per page (paged tiers) and per code block (compact tier). */
 #define AKV_PAGE_TOKENS 16
 
-/* Bytes of one compact-tier block of 16 tokens for head dim d: 16 code rows of d/2 bytes
- * (token order; byte k of a row holds code 2k in its low nibble and code 2k+1 in its
- * high nibble), then 16 little-endian binary16 scales.  1056 bytes at d = 128. */
+/* Bytes of one compact-tier block of 16 tokens for head dim d, then 16 little-endian
+ * binary16 scales; 1056 bytes at d = 128.
+ *   Key blocks: 16 code rows of d/2 bytes (token order; byte k of a row holds code 2k in
+ *   its low nibble and code 2k+1 in its high nibble).
+ *   Value blocks: 8 pair rows of d bytes; byte k of pair row r holds code k of token 2r in
+ *   its low nibble and code k of token 2r+1 in its high nibble; the d bytes of pair row r
+ *   are 8 units of d/8 bytes with unit u stored at position u ^ w(r), w(r) = 2 (r % 4)
+ *   for d = 128 and 4 ((r / 2) % 2) for d = 64 (the tensor-core operand order, read
+ *   without bank conflicts).
+ * akv_encode_history writes both; other producers must follow the same layout. */
 #define AKV_CODES4_BLOCK_BYTES(d) (16 * ((d) / 2) + 32)
 
 /*
@@ -102,8 +112,8 @@ enum { AKV_TIER_BF16 = 0, AKV_TIER_CODES4 = 1 };
  *   BF16, paged:        k + P*stride_seq + h*stride_head + (t%16)*stride_token,
  *                       P = page_table[b*page_table_stride + t/16]               (elements)
  *   CODES4, contiguous: block k + b*stride_seq + h*stride_head + (t/16)*stride_token,
- *                       row t%16 of that block                                   (blocks)
- *   CODES4, paged:      block k + P*stride_seq + h*stride_head, row t%16         (blocks)
+ *                       token t%16 of that block                                 (blocks)
+ *   CODES4, paged:      block k + P*stride_seq + h*stride_head, token t%16       (blocks)
  * The head dimension is contiguous.  V uses the same layout from base v.
  * BF16 bases must be 16-byte aligned and BF16 strides multiples of 8 elements; CODES4
  * bases must be 16-byte aligned.  Buffers must cover every addressed token: the library

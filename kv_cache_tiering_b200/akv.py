@@ -25,11 +25,13 @@ AKV_ERR_TIMEOUT = -6
 AKV_ERR_NONFINITE = -7
 AKV_ERR_RANGE = -8
 AKV_ERR_BOUNDS = -9
+AKV_ERR_INTERNAL = -10
 
 AKV_EFLAG_NONFINITE = 0x1
 AKV_EFLAG_RANGE = 0x2
 AKV_EFLAG_BOUNDS = 0x4
 AKV_EFLAG_TIMEOUT = 0x8
+AKV_EFLAG_INTERNAL = 0x10
 
 AKV_TIER_BF16 = 0
 AKV_TIER_CODES4 = 1

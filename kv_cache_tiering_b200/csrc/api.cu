@@ -215,11 +215,13 @@ const char* akv_status_string(int status) {
     case AKV_ERR_NONFINITE: return "non-finite input";
     case AKV_ERR_RANGE: return "norm out of binary16 range";
     case AKV_ERR_BOUNDS: return "page id out of bounds";
+    case AKV_ERR_INTERNAL: return "kernel launch configuration defect";
     default: return "unknown status";
   }
 }
 
 akv_status akv_error_word_status(int32_t word) {
+  if (word & AKV_EFLAG_INTERNAL) return AKV_ERR_INTERNAL;
   if (word & AKV_EFLAG_TIMEOUT) return AKV_ERR_TIMEOUT;
   if (word & AKV_EFLAG_BOUNDS) return AKV_ERR_BOUNDS;
   if (word & AKV_EFLAG_NONFINITE) return AKV_ERR_NONFINITE;

@@ -101,19 +101,56 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
+// The MMAs are plain asm: their results depend only on their operands, so the compiler may
+// interleave them with independent work.
 __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Shared-memory loads on 32-bit shared-window addresses, with an immediate offset.  Ring
+// stages are read with volatile asm, which keeps each read after the cp.async wait that
+// publishes the stage; table reads are plain, the table being constant once built.
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1+%2];\n" : "=r"(v) : "r"(a), "n"(OFF));
+  return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2+%3];\n" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
+  return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4+%5];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a), "n"(OFF));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32_const(uint32_t a) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(a));
+  return v;
+}
+// 2^x on the special-function unit (ex2.approx: relative error about 2^-22, -inf -> +0,
+// subnormal results flushed to zero).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -201,8 +238,8 @@ __device__ __forceinline__ void cursor_next(const AttendParams& p, Cursor& c, in
 // head c % 4 for G <= 4).  Returns false when no rescale is needed (all factors 1, or the
 // chain's first step, whose accumulators are still zero).
 // ------------------------------------------------------------------------------------
-template <int G>
-__device__ __forceinline__ bool online_softmax(float (&sc)[2][4], float& m_run, float& l_run, float& a_even,
+template <int G, int N>
+__device__ __forceinline__ bool online_softmax(float (&sc)[2][N], float& m_run, float& l_run, float& a_even,
                                                float& a_odd) {
   const int lane = threadIdx.x & 31, tq = lane & 3;
   float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
@@ -210,13 +247,13 @@ __device__ __forceinline__ bool online_softmax(float (&sc)[2][4], float& m_run, 
   mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
   const float m_new = fmaxf(m_run, mx);
   const bool grow = m_new > m_run && m_run != -INFINITY;  // a chain's first step has nothing to rescale
-  const float alpha = exp2f(m_run - m_new);  // 0 on a chain's first step (m_run = -inf)
+  const float alpha = fast_exp2(m_run - m_new);  // 0 on a chain's first step (m_run = -inf)
   float s = 0.f;
 #pragma unroll
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      sc[j][e] = exp2f(sc[j][e] - m_new);
+      sc[j][e] = fast_exp2(sc[j][e] - m_new);
       s += sc[j][e];
     }
   l_run = l_run * alpha + s;
@@ -614,51 +651,74 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
 // Every split of the compact tier is one chain: a single warp runs all of its 16-token
 // steps in order, so the split needs no cross-warp merge.  The grid is persistent (one CTA
 // of NWARP warps per SM) and every warp owns an equal contiguous range of items.
-// Shared memory: the lookup table, 256 rows of 256 bytes (entry b for lane l at byte
-// 256 b + 4 l: the half pair (c[b & 15], c[b >> 4]); one copy per lane keeps the gathers
-// conflict-free, and the row stride lets one byte permute build the address); then per
-// warp a scratch of G x D words (query rotation, output rotation) and a ring of NST
-// stages.  A stage holds one 16-token block of K (its own layout: code rows, then 16
-// scales) and of V (code rows padded to VROW bytes so the four token lanes' reads fall in
-// different banks, then 16 scales), filled by cp.async.
+//
+// Shared memory.  The lookup table is 256 rows of 256 bytes at the first 64 KB boundary of
+// the CTA's window: entry b for lane l sits at table + 256 b + 4 l and holds the half pair
+// (c[b & 15], c[b >> 4]).  One copy per lane keeps the gathers conflict-free, and with the
+// table 64 KB aligned one byte permute of (code word, table | 4 lane) yields the entry's
+// full shared address.  The upper 128 bytes of every table row are each warp's scratch
+// (G x D words for the query and output rotations, SCR_ROWS rows per warp).  Each warp's
+// ring of NST stages sits below the table while they fit and above it after.  A stage
+// holds one 16-token key block and one value block exactly as stored, filled by cp.async.
+// The value block's pair-row layout (byte k of pair row r = code k of tokens 2r, 2r + 1;
+// unit u of D/8 bytes at position u ^ w(r)) is the A-fragment order of the value product,
+// and its unit swizzle makes the fragment reads conflict-free.
 template <int D, int G, int NWARP, int NST>
 struct CodesCfg {
   static constexpr int ROWB = D / 2;
-  static constexpr int VROW = ROWB + 16;
-  static constexpr int K_OFF = 0;
-  static constexpr int KS_OFF = 16 * ROWB;
-  static constexpr int V_OFF = KS_OFF + 32;
-  static constexpr int VS_OFF = V_OFF + 16 * VROW;
-  static constexpr int STAGE = VS_OFF + 32;
   static constexpr int BLOCK = AKV_CODES4_BLOCK_BYTES(D);
-  static constexpr int LUT = 256 * 256;
-  static constexpr int SCRATCH = (G * D + 16) * 4;  // words, plus per-head scales
-  static constexpr int PER_WARP = SCRATCH + NST * STAGE;
-  static constexpr size_t SMEM = (size_t)LUT + (size_t)NWARP * PER_WARP;
+  static constexpr int K_OFF = 0;                  // the key block as stored
+  static constexpr int KS_OFF = 16 * ROWB;
+  static constexpr int V_OFF = BLOCK;              // the value block as stored
+  static constexpr int VS_OFF = BLOCK + 16 * ROWB;
+  static constexpr int US = D / 8;                 // value unit: one lane group's dims
+  static constexpr int STAGE = 2 * BLOCK;
+  static constexpr int LUT = 1 << 16;
+  static constexpr int SCR_ROWS = G * D / 32;
+  static constexpr int PER_WARP = NST * STAGE;
+  // Wherever the window starts, the rings below the table waste less than one ring, and
+  // an all-below layout ends within two table lengths of the start.
+  static constexpr int SPAN = NWARP * PER_WARP + PER_WARP;
+  static constexpr size_t SMEM = (size_t)LUT + (size_t)(SPAN > LUT ? SPAN : LUT);
+  static_assert(SCR_ROWS * NWARP <= 256, "scratch fits the table rows' upper halves");
+  static_assert(PER_WARP % 16 == 0 && STAGE % 16 == 0, "16-byte aligned rings and stages");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
+
+// Where the table and this warp's ring sit; false when the launch's dynamic shared memory
+// is too small for the layout (the caller flags it and does nothing).
+template <class C, int NWARP>
+__device__ __forceinline__ bool codes_layout(uint32_t base_s, int warp, uint32_t& lut_s, uint32_t& ring_s) {
+  lut_s = (base_s + 0xFFFFu) & ~0xFFFFu;
+  const int below = min(NWARP, (int)((lut_s - base_s) / C::PER_WARP));
+  const uint32_t top = lut_s + C::LUT + (uint32_t)(NWARP - below) * C::PER_WARP;
+  uint32_t dyn;
+  asm("mov.u32 %0, %%dynamic_smem_size;\n" : "=r"(dyn));
+  ring_s = warp < below ? base_s + warp * C::PER_WARP : lut_s + C::LUT + (warp - below) * C::PER_WARP;
+  return top - base_s <= dyn;
+}
+
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
+}
 
 template <int D, int G, int NWARP, int NST>
 __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_constant__ AttendParams p) {
   using C = CodesCfg<D, G, NWARP, NST>;
   constexpr int DPT = D / 8;                      // value dims per lane group
   constexpr int KB = D / 8;                       // key code bytes per lane
-  constexpr int NWD = DPT / 8 > 0 ? DPT / 8 : 1;  // value code words per token per lane
   constexpr int P = D / 32;                       // coordinates per lane in a warp-wide row
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  uint8_t* wbase = smem + C::LUT + (size_t)warp * C::PER_WARP;
-  uint32_t* scratch = reinterpret_cast<uint32_t*>(wbase);   // [G][D] words
-  float* scratchf = reinterpret_cast<float*>(wbase);
-  float* hscale = reinterpret_cast<float*>(wbase) + G * D;  // [G]
-  uint8_t* ring = wbase + C::SCRATCH;
-  const uint32_t ring_s = smem_u32(ring);
-
-  for (int i = threadIdx.x; i < 256 * 32; i += NWARP * 32) {
-    const int byte = i >> 5, l = i & 31;
-    lut[byte * 64 + l] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
+  const uint32_t base_s = smem_u32(smem);
+  uint32_t lut_s, ring_s;
+  if (!codes_layout<C, NWARP>(base_s, warp, lut_s, ring_s)) {  // same answer in every thread
+    if (threadIdx.x == 0) flag_error(p.err, AKV_EFLAG_INTERNAL);
+    return;
   }
-  __syncthreads();
+  // word i of this warp's scratch: word i % 32 of the upper half of its table row i / 32
+  const uint32_t scr_s = lut_s + (uint32_t)(warp * C::SCR_ROWS) * 256u + 128u;
+  auto scr = [&](int i) -> uint32_t { return scr_s + ((uint32_t)(i >> 5) << 8) + ((uint32_t)(i & 31) << 2); };
 
   // this warp's item range: an equal share of all items, in item order; warps are numbered
   // warp-major across CTAs so a partly filled grid still spreads its busy warps over every SM
@@ -666,110 +726,199 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   const int nw = (int)gridDim.x * NWARP, gw = warp * (int)gridDim.x + (int)blockIdx.x;
   const int q0 = total / nw, r0 = total % nw;
   const int lo = gw * q0 + min(gw, r0), hi = lo + q0 + (gw < r0 ? 1 : 0);
-  if (lo >= hi) return;
+  const bool busy = lo < hi;
 
-  // stage fill through cp.async 16-byte chunks: lane l copies code chunks l and l + 32 of K
-  // (the block's own layout) and of V (into the padded rows); lanes 0 and 1 also copy the
-  // two scale chunks of each
-  constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per code row
-  constexpr bool kTwo = C::ROWB > 32;
-  const uint32_t kd0 = C::K_OFF + 16 * lane, kd1 = kd0 + 16 * 32;
-  const uint32_t vd0 = C::V_OFF + (lane / CPR) * C::VROW + 16 * (lane % CPR);
-  const uint32_t vd1 = C::V_OFF + ((lane + 32) / CPR) * C::VROW + 16 * ((lane + 32) % CPR);
-  auto load_step = [&](const Item& it, int s, int st) {
-    const int tok0 = it.t0 + 16 * s;
-    int64_t blk;
-    if (p.tier.paged) {
-      blk = tier_page(p.tier, it.b, tok0 >> 4, p.err) * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head;
-    } else {
-      blk = (int64_t)it.b * p.tier.s_seq + (int64_t)it.kvh * p.tier.s_head + (int64_t)(tok0 >> 4) * p.tier.s_tok;
+  // the query rows of an item's G heads, P bf16 coordinates per lane each, one load per head;
+  // the first item's are requested before anything else so their latency hides behind the
+  // stage loads and the table build
+  auto load_q = [&](const Item& it, uint32_t (&qw)[G][P / 2]) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint16_t* qrow = p.q + ((size_t)it.b * p.Hq + (size_t)it.kvh * G + h) * D + P * lane;
+      if constexpr (P == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(qrow);
+        qw[h][0] = v.x;
+        qw[h][1] = v.y;
+      } else {
+        qw[h][0] = *reinterpret_cast<const uint32_t*>(qrow);
+      }
     }
+  };
+  uint32_t qw[G][P / 2];
+  if (busy) load_q(item_at(p, lo), qw);
+
+  // ---- loader: the (item, step) of the next stage to fill.  Global step S of this warp
+  // (counted over its items) uses stage S % NST.  The lanes copy the key block and the value
+  // block into it as stored, in 16-byte chunks (lane l: chunks l, l + 32, l + 64 of each
+  // that exist), as one cp.async commit group per step.
+  constexpr int CH = C::BLOCK / 16;  // 16-byte chunks per block
+  static_assert(CH > 32 && CH <= 96, "at most three chunk rounds per block");
+  int ld_item = lo, ld_left = 0;  // the loader's item and its steps not yet issued
+  int ld_b = 0, ld_lp = 0;         // its sequence and the logical page of its next step
+  int64_t ld_blk = 0;              // contiguous: block of the next step; paged: the head's offset
+  auto ld_begin = [&]() {
+    const Item it = item_at(p, ld_item);
+    ld_left = (it.n + 15) >> 4;
+    ld_b = it.b;
+    ld_lp = it.t0 >> 4;
+    ld_blk = (int64_t)it.kvh * p.tier.s_head;
+    if (!p.tier.paged) ld_blk += (int64_t)it.b * p.tier.s_seq + (int64_t)ld_lp * p.tier.s_tok;
+  };
+  auto ld_issue = [&](int stage) {
+    int64_t blk = ld_blk;
+    if (p.tier.paged) {
+      blk += tier_page(p.tier, ld_b, ld_lp, p.err) * p.tier.s_seq;
+    } else {
+      ld_blk += p.tier.s_tok;
+    }
+    const uint32_t dst = ring_s + stage * C::STAGE + 16 * lane;
     const uint8_t* kb = p.tier.k + blk * C::BLOCK + 16 * lane;
     const uint8_t* vb = p.tier.v + blk * C::BLOCK + 16 * lane;
-    const uint32_t dst = ring_s + st * C::STAGE;
-    cp_async16(dst + kd0, kb);
-    cp_async16(dst + vd0, vb);
-    if constexpr (kTwo) {
-      cp_async16(dst + kd1, kb + 16 * 32);
-      cp_async16(dst + vd1, vb + 16 * 32);
+    cp_async16(dst + C::K_OFF, kb);
+    cp_async16(dst + C::V_OFF, vb);
+    if (CH >= 64 || 32 + lane < CH) {
+      cp_async16(dst + C::K_OFF + 512, kb + 512);
+      cp_async16(dst + C::V_OFF + 512, vb + 512);
     }
-    if (lane < 2) {
-      cp_async16(dst + C::KS_OFF + 16 * lane, kb + 16 * C::ROWB);
-      cp_async16(dst + C::VS_OFF + 16 * lane, vb + 16 * C::ROWB);
+    if (64 + lane < CH) {
+      cp_async16(dst + C::K_OFF + 1024, kb + 1024);
+      cp_async16(dst + C::V_OFF + 1024, vb + 1024);
     }
+    ++ld_lp;
+    if (--ld_left == 0 && ++ld_item < hi) ld_begin();
   };
-
-  // cursor over (item, step): all steps of each item in order
-  Cursor ld;
-  ld.item = lo;
-  ld.step = 0;
-  ld.info = item_at(p, ld.item);
+  if (busy) {
+    ld_begin();
 #pragma unroll
-  for (int j = 0; j < NST; ++j) {
-    if (ld.item < hi) {
-      load_step(ld.info, ld.step, j);
-      cursor_next<1, 1>(p, ld, hi, 0);
+    for (int j = 0; j < NST; ++j) {
+      if (ld_item < hi) ld_issue(j);
+      cp_async_commit();
     }
-    cp_async_commit();
   }
 
-  // table address of byte `byte` of `word` for this lane: (word.byte << 8) | (lane << 2)
-  const uint32_t lane4 = (uint32_t)lane << 2;
+  {
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_s - base_s));
+    for (int i = threadIdx.x; i < 256 * 32; i += NWARP * 32) {
+      const int byte = i >> 5, l = i & 31;
+      lut[byte * 64 + l] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
+    }
+  }
+  __syncthreads();
+  if (!busy) return;
+
+  // table entry of byte `byte` of `word` for this lane: the table's own high address bytes,
+  // the code byte as bits 8..15 and 4 lane as bits 0..7, assembled by one byte permute
+  const uint32_t lane4 = lut_s | ((uint32_t)lane << 2);
   auto lookup = [&](uint32_t word, int byte) -> uint32_t {
-    const uint32_t addr = __byte_perm(word, lane4, 0x5504 | (byte << 4));
-    return *reinterpret_cast<const uint32_t*>(smem + addr);
+    return lds32_const(__byte_perm(word, lane4, 0x7604 | (byte << 4)));
   };
+  // this lane's offsets inside a stage: key code bytes [KB tq, KB tq + KB) of token g (+ 8),
+  // the scales of tokens 2tq, 2tq + 1 (+ 8), value code bytes of dims [DPT g, DPT g + DPT)
+  // of tokens 2tq, 2tq + 1 (+ 8)
+  const uint32_t koff = C::K_OFF + g * C::ROWB + KB * tq;
+  const uint32_t ksoff = C::KS_OFF + 4 * tq;  // the value scales sit at + VS_OFF - KS_OFF
+  const uint32_t voff = C::V_OFF + tq * D + C::US * (g ^ (D == 128 ? 2 * tq : 4 * (tq >> 1)));
+  static_assert((NST & (NST - 1)) == 0, "stage index by mask");
+  int gs = 0;  // this warp's global step; its stage is gs % NST
 
   uint32_t qa[D / 16][4];
   float kfac = 0.f;
   int q_pair = -1;
-  int stage = 0;
+
+  // Base-2 scores of the step held in stage sa: sc[j][e] is head g at token 8j + 2tq + e,
+  // S^T = (H q) K_hat^T with the B fragments looked up straight from the code bytes, the
+  // high (row g) and residual (row g + 8) parts added, times the key scale.
+  auto scores = [&](uint32_t sa, float (&sc)[2][2]) {
+    uint32_t wk[2][KB / 4];
+    const uint32_t ka = sa + koff;
+    if constexpr (KB == 16) {
+      const uint4 a = lds128<0>(ka), b = lds128<8 * C::ROWB>(ka);
+      wk[0][0] = a.x; wk[0][1] = a.y; wk[0][2] = a.z; wk[0][3] = a.w;
+      wk[1][0] = b.x; wk[1][1] = b.y; wk[1][2] = b.z; wk[1][3] = b.w;
+    } else {
+      const uint2 a = lds64<0>(ka), b = lds64<8 * C::ROWB>(ka);
+      wk[0][0] = a.x; wk[0][1] = a.y;
+      wk[1][0] = b.x; wk[1][1] = b.y;
+    }
+    float st[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[j][e] = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < D / 16; ++kc)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t wd = wk[j][kc >> 1];
+        mma_f16(st[j], qa[kc], lookup(wd, 2 * (kc & 1)), lookup(wd, 2 * (kc & 1) + 1));
+      }
+    const uint32_t ksw[2] = {lds32<0>(sa + ksoff), lds32<16>(sa + ksoff)};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float2 kh = unpack_f16(ksw[j]);
+      sc[j][0] = (st[j][0] + st[j][2]) * (kfac * kh.x);
+      sc[j][1] = (st[j][1] + st[j][3]) * (kfac * kh.y);
+    }
+  };
 
   for (int item = lo; item < hi; ++item) {
     const Item it = item_at(p, item);
     if (it.pair != q_pair) {
+      if (item != lo) load_q(it, qw);
       q_pair = it.pair;
-      // rotate each head: H q by shuffles, a power-of-two scale to [0.5, 1), then the
-      // FP16 (high, residual) words of dims (P*lane + j, P*lane + j + 1) into the scratch
-      __syncwarp();
-#pragma unroll 1
+      // rotate the heads together: H q by shuffles, a power-of-two scale to [0.5, 1), then
+      // the FP16 (high, residual) words of dims (P*lane + j, P*lane + j + 1) into the scratch
+      float x[G][P];
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int j = 0; j < P / 2; ++j) {
+          x[h][2 * j] = bf16lo(qw[h][j]);
+          x[h][2 * j + 1] = bf16hi(qw[h][j]);
+        }
+#pragma unroll
+      for (int h = 0; h < G; ++h) warp_fwht<P>(x[h]);
+      float mx[G];
+#pragma unroll
       for (int h = 0; h < G; ++h) {
-        const uint16_t* qrow = p.q + ((size_t)it.b * p.Hq + (size_t)it.kvh * G + h) * D + P * lane;
-        float x[P];
+        mx[h] = 0.f;
 #pragma unroll
-        for (int j = 0; j < P; ++j) x[j] = bf16_to_float(qrow[j]);
-        warp_fwht<P>(x);
-        float mx = 0.f;
+        for (int j = 0; j < P; ++j) mx[h] = fmaxf(mx[h], fabsf(x[h][j]));
+      }
 #pragma unroll
-        for (int j = 0; j < P; ++j) mx = fmaxf(mx, fabsf(x[j]));
+      for (int off = 16; off >= 1; off >>= 1)
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], off));
+      __syncwarp();  // earlier reads of the scratch are done
+      int my_e = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
         int e = 0;
-        if (mx > 0.f) frexpf(mx, &e);
+        if (mx[h] > 0.f) frexpf(mx[h], &e);
         const float inv = ldexpf(1.f, -e);
 #pragma unroll
         for (int j = 0; j < P; j += 2) {
-          const float x0 = x[j] * inv, x1 = x[j + 1] * inv;
+          const float x0 = x[h][j] * inv, x1 = x[h][j + 1] * inv;
           const uint32_t hw = pack_f16(x0, x1);
           const float2 hv = unpack_f16(hw);
-          scratch[h * D + P * lane + j] = hw;
-          scratch[h * D + P * lane + j + 1] = pack_f16(x0 - hv.x, x1 - hv.y);
+          sts32(scr(h * D + P * lane + j), hw);
+          sts32(scr(h * D + P * lane + j + 1), pack_f16(x0 - hv.x, x1 - hv.y));
         }
-        if (lane == 0) hscale[h] = ldexpf(1.f, e);
+        if (g == h) my_e = e;
       }
       __syncwarp();
       // lane (g, tq), step kc covers dims 2*KB*tq + 4kc + {0,1,2,3}: rows g = high parts,
       // rows g + 8 = residuals
-      const int h = g < G ? g : 0;
-      const uint32_t* qrow = scratch + h * D + 2 * KB * tq;
+      const int i0 = (g < G ? g : 0) * D + 2 * KB * tq;
 #pragma unroll
       for (int kc = 0; kc < D / 16; ++kc) {
-        qa[kc][0] = g < G ? qrow[4 * kc] : 0u;       // high, dims 4kc, 4kc+1
-        qa[kc][1] = g < G ? qrow[4 * kc + 1] : 0u;   // residual
-        qa[kc][2] = g < G ? qrow[4 * kc + 2] : 0u;   // high, dims 4kc+2, 4kc+3
-        qa[kc][3] = g < G ? qrow[4 * kc + 3] : 0u;   // residual
+        const uint4 v = lds128<0>(scr(i0 + 4 * kc));
+        qa[kc][0] = g < G ? v.x : 0u;  // high, dims 4kc, 4kc+1
+        qa[kc][1] = g < G ? v.y : 0u;  // residual
+        qa[kc][2] = g < G ? v.z : 0u;  // high, dims 4kc+2, 4kc+3
+        qa[kc][3] = g < G ? v.w : 0u;  // residual
       }
-      kfac = p.scale_log2 / (float)D * hscale[h];
+      kfac = p.scale_log2 / (float)D * ldexpf(1.f, my_e);
       __syncwarp();
     }
 
@@ -779,48 +928,22 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;
+    const int nsteps = (it.n + 15) >> 4;
+    // Commit groups are counted in steps: before step S of this warp NST + S groups have been
+    // committed, so waiting down to NST - 1 pending lands step S, and down to NST - 2 lands
+    // step S + 1 as well.
+    float sc_n[2][2];
+    cp_async_wait<NST - 1>();
+    __syncwarp();
+    scores(ring_s + (gs & (NST - 1)) * C::STAGE, sc_n);
 
-    for (int s = 0; 16 * s < it.n; ++s) {
-      cp_async_wait<NST - 1>();
+    for (int s = 0; s < nsteps; ++s) {
+      cp_async_wait<NST - 2>();  // this step and the next have landed
       __syncwarp();
+      const uint32_t st_s = ring_s + (gs & (NST - 1)) * C::STAGE;
+      const uint32_t nxt = ring_s + ((gs + 1) & (NST - 1)) * C::STAGE;
+      float sc[2][2] = {{sc_n[0][0], sc_n[0][1]}, {sc_n[1][0], sc_n[1][1]}};
       const int nv = min(16, it.n - 16 * s);
-      const uint8_t* sk = ring + stage * C::STAGE;
-      // ---- S^T = (H q) K_hat^T: B fragments straight from the code bytes
-      float sc[2][4];
-      uint32_t wk[2][KB / 4];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[j][e] = 0.f;
-        const uint8_t* row = sk + C::K_OFF + (8 * j + g) * C::ROWB + KB * tq;
-        if constexpr (KB == 16) {
-          const uint4 v = *reinterpret_cast<const uint4*>(row);
-          wk[j][0] = v.x; wk[j][1] = v.y; wk[j][2] = v.z; wk[j][3] = v.w;
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2*>(row);
-          wk[j][0] = v.x; wk[j][1] = v.y;
-        }
-      }
-#pragma unroll
-      for (int kc = 0; kc < D / 16; ++kc)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t wd = wk[j][kc >> 1];
-          mma_f16(sc[j], qa[kc], lookup(wd, 2 * (kc & 1)), lookup(wd, 2 * (kc & 1) + 1));
-        }
-      float ksc[2][2], vsc[2][2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float2 kh = unpack_f16(*reinterpret_cast<const uint32_t*>(sk + C::KS_OFF + 2 * (8 * j + 2 * tq)));
-        const float2 vh = unpack_f16(*reinterpret_cast<const uint32_t*>(sk + C::VS_OFF + 2 * (8 * j + 2 * tq)));
-        ksc[j][0] = kh.x; ksc[j][1] = kh.y;
-        vsc[j][0] = vh.x; vsc[j][1] = vh.y;
-      }
-      // score of head g = high row g + residual row g + 8
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) sc[j][e] = (sc[j][e] + sc[j][e + 2]) * (kfac * ksc[j][e]);
       if (nv < 16) {
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -828,6 +951,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
           for (int e = 0; e < 2; ++e)
             if (8 * j + 2 * tq + e >= nv) sc[j][e] = -INFINITY;
       }
+      // the next step's scores, so their loads, lookups and MMAs overlap this step's
+      // softmax and value product (after an item's last step the next stage holds the
+      // following item's first step or nothing; those scores are not used)
+      scores(nxt, sc_n);
       float a_even, a_odd;
       if (online_softmax<G>(sc, m_run, l_run, a_even, a_odd)) {
 #pragma unroll
@@ -837,11 +964,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         }
       }
       // ---- P' = P * s^V (0 for masked tokens): FP16 high part and residual
+      const uint32_t vsw[2] = {lds32<C::VS_OFF - C::KS_OFF>(st_s + ksoff),
+                               lds32<C::VS_OFF - C::KS_OFF + 16>(st_s + ksoff)};
       float wts[2][2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) wts[j][e] = sc[j][e] * vsc[j][e];
+      for (int j = 0; j < 2; ++j) {
+        const float2 vh = unpack_f16(vsw[j]);
+        wts[j][0] = sc[j][0] * vh.x;
+        wts[j][1] = sc[j][1] * vh.y;
+      }
       if (nv < 16) {
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -851,47 +982,35 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       }
       uint32_t pb[2], pl[2];
       p_fragments<G, false>(wts, pb, pl);
-      // ---- O_rot^T += V_hat^T P'^T: lane (g, tq) supplies value dims [DPT g, DPT g + DPT)
-      // of tokens (2tq, 2tq+1) and (2tq+8, 2tq+9); one byte = the nibbles of two tokens
-      uint32_t z[2][NWD][2];
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        const uint8_t* r0 = sk + C::V_OFF + (8 * pr + 2 * tq) * C::VROW + (DPT / 2) * g;
-        const uint8_t* r1 = r0 + C::VROW;
-        uint32_t w0[NWD], w1[NWD];
-        if constexpr (NWD == 2) {
-          const uint2 a = *reinterpret_cast<const uint2*>(r0);
-          const uint2 b = *reinterpret_cast<const uint2*>(r1);
-          w0[0] = a.x; w0[1] = a.y; w1[0] = b.x; w1[1] = b.y;
-        } else {
-          w0[0] = *reinterpret_cast<const uint32_t*>(r0);
-          w1[0] = *reinterpret_cast<const uint32_t*>(r1);
-        }
-#pragma unroll
-        for (int wi = 0; wi < NWD; ++wi) {
-          z[pr][wi][0] = (w0[wi] & 0x0F0F0F0Fu) | ((w1[wi] & 0x0F0F0F0Fu) << 4);
-          z[pr][wi][1] = ((w0[wi] >> 4) & 0x0F0F0F0Fu) | (w1[wi] & 0xF0F0F0F0u);
-        }
+      // ---- O_rot^T += V_hat^T P'^T: lane (g, tq) reads value dims [DPT g, DPT g + DPT) of
+      // token pairs (2tq, 2tq+1) (pair row tq) and (2tq+8, 2tq+9) (pair row 4 + tq); byte k
+      // of those words is dim DPT g + k of both tokens, so one lookup is one A-fragment entry
+      uint32_t vw[2][DPT / 4];
+      const uint32_t va = st_s + voff;
+      if constexpr (DPT == 16) {
+        const uint4 a = lds128<0>(va), b = lds128<4 * D>(va);
+        vw[0][0] = a.x; vw[0][1] = a.y; vw[0][2] = a.z; vw[0][3] = a.w;
+        vw[1][0] = b.x; vw[1][1] = b.y; vw[1][2] = b.z; vw[1][3] = b.w;
+      } else {
+        const uint2 a = lds64<0>(va), b = lds64<4 * D>(va);
+        vw[0][0] = a.x; vw[0][1] = a.y;
+        vw[1][0] = b.x; vw[1][1] = b.y;
       }
-      // dim offset m lives in word m / 8, byte (m % 8) / 2, parity m % 2
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) {
         uint32_t a[4];
-        const int m0 = mt, m1 = DPT / 2 + mt;
-        a[0] = lookup(z[0][m0 >> 3][m0 & 1], (m0 & 7) >> 1);
-        a[1] = lookup(z[0][m1 >> 3][m1 & 1], (m1 & 7) >> 1);
-        a[2] = lookup(z[1][m0 >> 3][m0 & 1], (m0 & 7) >> 1);
-        a[3] = lookup(z[1][m1 >> 3][m1 & 1], (m1 & 7) >> 1);
+        const int m0 = mt, m1 = DPT / 2 + mt;  // rows g and g + 8 of this 16-dim tile
+        a[0] = lookup(vw[0][m0 >> 2], m0 & 3);
+        a[1] = lookup(vw[0][m1 >> 2], m1 & 3);
+        a[2] = lookup(vw[1][m0 >> 2], m0 & 3);
+        a[3] = lookup(vw[1][m1 >> 2], m1 & 3);
         mma_f16(acc[mt], a, pb[0], pb[1]);
         if constexpr (G > 4) mma_f16(acc[mt], a, pl[0], pl[1]);
       }
       __syncwarp();
-      if (ld.item < hi) {
-        load_step(ld.info, ld.step, stage);
-        cursor_next<1, 1>(p, ld, hi, 0);
-      }
+      if (ld_item < hi) ld_issue(gs & (NST - 1));  // refills the stage just read
       cp_async_commit();
-      stage = stage + 1 == NST ? 0 : stage + 1;
+      ++gs;
     }
 
     // ---- epilogue: O = H (acc / l) / D per head, LSE = ln 2 (m + log2 l)
@@ -916,14 +1035,20 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       for (int e = 0; e < 4; ++e) {
         const int h = 2 * tq + (e & 1);
         const int dim = DPT * g + ((e >> 1) ? DPT / 2 : 0) + mt;
-        if (h < G) scratchf[h * D + dim] = acc[mt][e] * ((e & 1) ? f_odd : f_even);
+        if (h < G) sts32(scr(h * D + dim), __float_as_uint(acc[mt][e] * ((e & 1) ? f_odd : f_even)));
       }
     __syncwarp();
-#pragma unroll 1
+#pragma unroll
     for (int h = 0; h < G; ++h) {
       float x[P];
-#pragma unroll
-      for (int j = 0; j < P; ++j) x[j] = scratchf[h * D + P * lane + j];
+      if constexpr (P == 4) {
+        const uint4 v = lds128<0>(scr(h * D + P * lane));
+        x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+        x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+      } else {
+        const uint2 v = lds64<0>(scr(h * D + P * lane));
+        x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+      }
       warp_fwht<P>(x);
       float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
       if constexpr (P == 4) {
@@ -972,7 +1097,7 @@ cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s) {
 template <int D, int G>
 cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
   constexpr int NWARP = G <= 4 ? 16 : 8;
-  constexpr int NST = 3;
+  constexpr int NST = 4;
   using C = CodesCfg<D, G, NWARP, NST>;
   auto k = attend_codes_mma<D, G, NWARP, NST>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);

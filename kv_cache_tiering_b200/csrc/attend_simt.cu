@@ -286,6 +286,23 @@ __global__ void __launch_bounds__(kThreads) attend_bf16_simt(const __grid_consta
 // ------------------------------------------------------------------------------------
 // compact tier (CODES4)
 // ------------------------------------------------------------------------------------
+// Value codes of dims col .. col + 7 (col a multiple of 8) of token t of a value block, in
+// the key row layout (byte j = dims col + 2j, col + 2j + 1).  A value block stores token
+// pairs: byte k of pair row r holds dim k of tokens 2r and 2r + 1, units of D/8 bytes at
+// position u ^ w(r).
+template <int D>
+__device__ __forceinline__ uint32_t value_codes8(const uint8_t* blk, int t, int col) {
+  constexpr int US = D / 8;
+  const int r = t >> 1;
+  const int w = D == 128 ? 2 * (r & 3) : 4 * ((r >> 1) & 1);
+  const uint2 v = *reinterpret_cast<const uint2*>(blk + r * D + ((col / US) ^ w) * US + col % US);
+  const int sh = 4 * (t & 1);
+  uint32_t x = (v.x >> sh) & 0x0F0F0F0Fu, y = (v.y >> sh) & 0x0F0F0F0Fu;
+  x |= x >> 4;  // bytes 0 and 2 now hold dim pairs (0, 1) and (2, 3)
+  y |= y >> 4;
+  return __byte_perm(x, y, 0x6420);
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads) attend_codes_simt(const __grid_constant__ AttendParams p) {
   constexpr int LPT = D / 8;        // lanes per token: 8 coordinates = 4 code bytes each
@@ -388,7 +405,7 @@ __global__ void __launch_bounds__(kThreads) attend_codes_simt(const __grid_const
         if (tt < si.n) {
           const int tok = si.t0 + tt;
           const uint8_t* blk = codes_block<D>(p.tier, p.tier.v, si.b, si.kvh, tok, p.err);
-          cw[u] = *reinterpret_cast<const uint32_t*>(blk + (tok & 15) * ROWB + col / 2);
+          cw[u] = value_codes8<D>(blk, tok & 15, col);
           sv[u] = half_bits_to_float(*reinterpret_cast<const uint16_t*>(blk + 16 * ROWB + 2 * (tok & 15)));
         } else {
           cw[u] = 0x77777777u;

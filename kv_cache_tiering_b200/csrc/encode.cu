@@ -21,9 +21,11 @@
 namespace akv {
 namespace {
 
+// Encode one vector: its code row (D/2 bytes, code 2k in the low nibble of byte k) goes to
+// code_row, its binary16 scale to scale_slot.
 template <int D>
-__device__ __forceinline__ void encode_vector(const uint8_t* src_row, uint8_t* block, int row, bool valid,
-                                              const double* bound, int32_t* err) {
+__device__ __forceinline__ void encode_vector(const uint8_t* src_row, uint8_t* code_row, uint16_t* scale_slot,
+                                              bool valid, const double* bound, int32_t* err) {
   constexpr int P = D / 32;  // coordinates per lane: 4 (d = 128) or 2 (d = 64)
   const int lane = threadIdx.x & 31;
   double z[P];
@@ -99,16 +101,12 @@ __device__ __forceinline__ void encode_vector(const uint8_t* src_row, uint8_t* b
     if (s == 0.0 || refuse || !valid) c = 7;
     codes |= (uint32_t)c << (4 * i);
   }
-  uint8_t* code_row = block + row * (D / 2);
   if constexpr (P == 4) {
     *reinterpret_cast<uint16_t*>(code_row + 2 * lane) = (uint16_t)codes;
   } else {
     code_row[lane] = (uint8_t)codes;
   }
-  if (lane == 0) {
-    uint16_t sbits = (refuse || !valid) ? (uint16_t)0 : __half_as_ushort(s16);
-    *reinterpret_cast<uint16_t*>(block + 16 * (D / 2) + 2 * row) = sbits;
-  }
+  if (lane == 0) *scale_slot = (refuse || !valid) ? (uint16_t)0 : __half_as_ushort(s16);
 }
 
 template <int D>
@@ -130,8 +128,31 @@ __global__ void __launch_bounds__(512) encode_kernel(const __grid_constant__ Enc
   uint8_t* vblock = const_cast<uint8_t*>(codes_block<D>(p.dst, p.dst.v, b, h, tok0, p.err));
   const uint8_t* ksrc = valid ? bf16_row(p.src, p.src.k, b, h, tok, p.err) : nullptr;
   const uint8_t* vsrc = valid ? bf16_row(p.src, p.src.v, b, h, tok, p.err) : nullptr;
-  encode_vector<D>(ksrc, kblock, row, valid, bound, p.err);
-  encode_vector<D>(vsrc, vblock, row, valid, bound, p.err);
+  constexpr int ROWB = D / 2;
+  // keys: the block's own row layout; values: code rows staged here, then stored by token
+  // pairs (byte k of pair row r = code k of token 2r | code k of token 2r + 1 << 4) with
+  // unit u of d/8 bytes at position u ^ w(r) -- the order the tensor-core product reads
+  __shared__ __align__(16) uint8_t vrows[16 * ROWB];
+  encode_vector<D>(ksrc, kblock + row * ROWB, reinterpret_cast<uint16_t*>(kblock + 16 * ROWB) + row, valid, bound,
+                   p.err);
+  encode_vector<D>(vsrc, vrows + row * ROWB, reinterpret_cast<uint16_t*>(vblock + 16 * ROWB) + row, valid, bound,
+                   p.err);
+  __syncthreads();
+  // 8 pair rows of D bytes = 16 ROWB bytes; thread i writes 4 bytes of pair row i / (D/4)
+  constexpr int US = D / 8;
+  for (int i = threadIdx.x; i < 16 * ROWB / 4; i += blockDim.x) {
+    const int r = i / (D / 4), k0 = 4 * (i % (D / 4));  // dims k0 .. k0 + 3 of pair row r
+    const uint8_t* lo = vrows + (2 * r) * ROWB + k0 / 2;
+    const uint8_t* hi = vrows + (2 * r + 1) * ROWB + k0 / 2;
+    const uint32_t a = (uint32_t)lo[0] | ((uint32_t)lo[1] << 8);  // codes of dims k0..k0+3, token 2r
+    const uint32_t c = (uint32_t)hi[0] | ((uint32_t)hi[1] << 8);  // token 2r + 1
+    uint32_t out = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out |= (((a >> (4 * j)) & 15u) | (((c >> (4 * j)) & 15u) << 4)) << (8 * j);
+    const int w = D == 128 ? 2 * (r & 3) : 4 * ((r >> 1) & 1);
+    const int u = k0 / US;
+    *reinterpret_cast<uint32_t*>(vblock + r * D + (u ^ w) * US + k0 % US) = out;
+  }
 }
 
 }  // namespace

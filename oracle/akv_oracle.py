@@ -33,10 +33,15 @@ Readings where the pages are silent (the plainest reading the rest supports):
   * Code of coordinate i: the number of boundaries b_j = (c_j + c_{j+1}) / 2 with
     z_i > s * b_j (strict), so ties go to the lower level and a zero coordinate gets
     code 7.  s == 0 gives all codes 7.  Every s * b_j is exact in float64.
-  * Packing: byte k of a vector's code row holds code 2k in its low nibble and code
-    2k+1 in its high nibble.  A 16-token block stores the 16 code rows (token order)
-    followed by the 16 binary16 scales (little-endian); unused slots of a partial
-    block hold the zero-vector encoding (codes 7, scale 0).
+  * Packing (the pages fix no storage layout): byte k of a key code row holds code 2k
+    in its low nibble and code 2k+1 in its high nibble.  A 16-token key block stores
+    the 16 code rows (token order) followed by the 16 binary16 scales (little-endian);
+    unused slots of a partial block hold the zero-vector encoding (codes 7, scale 0).
+    A value block stores the same codes by token pairs instead -- byte k of pair row r
+    holds code k of token 2r (low nibble) and of token 2r + 1 (high nibble) -- with the
+    d bytes of pair row r cut into 8 units of d/8 bytes and unit u stored at position
+    u XOR w(r), w(r) = 2 (r mod 4) for d = 128 and 4 (floor(r / 2) mod 2) for d = 64;
+    then the 16 scales as for keys.  (This is the order the tensor-core product reads.)
   * Dequantisation: y_i = s * c[code_i] / sqrt(d) in the rotated domain,
     x_hat = H y / sqrt(d) in the original domain.
   * Softmax scale sigma is applied inside; LSE is the natural log of sum exp(scores);
@@ -189,6 +194,59 @@ def pack_blocks(codes, scale_bits) -> np.ndarray:
     rows = pack_codes(full_codes).reshape(nb, BLOCK_TOKENS * (d // 2))
     sc = full_scales.reshape(nb, BLOCK_TOKENS).astype("<u2").view(np.uint8)
     return np.concatenate([rows, sc], axis=1)
+
+
+def value_unit_swizzle(r: int, d: int) -> int:
+    """w(r): the position XOR of the units of value pair row r (8 units of d/8 bytes)."""
+    if d == 128:
+        return 2 * (r % 4)
+    if d == 64:
+        return 4 * ((r // 2) % 2)
+    raise ValueError("value blocks are defined for d = 64 and d = 128")
+
+
+def pack_value_blocks(codes, scale_bits) -> np.ndarray:
+    """Value-block layout of the codes uint8 [T, d] and scales uint16 [T] of one
+    (sequence, KV head) stream: uint8 [ceil(T / 16), block_bytes(d)]."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scale_bits = np.asarray(scale_bits, dtype=np.uint16)
+    t, d = codes.shape
+    nb = -(-t // BLOCK_TOKENS)
+    full_codes = np.full((nb * BLOCK_TOKENS, d), 7, dtype=np.uint8)
+    full_codes[:t] = codes
+    full_scales = np.zeros(nb * BLOCK_TOKENS, dtype=np.uint16)
+    full_scales[:t] = scale_bits
+    unit = d // 8
+    out = np.zeros((nb, block_bytes(d)), dtype=np.uint8)
+    for n in range(nb):
+        blk = full_codes[n * BLOCK_TOKENS:(n + 1) * BLOCK_TOKENS]
+        for r in range(BLOCK_TOKENS // 2):
+            pair = (blk[2 * r] | (blk[2 * r + 1] << 4)).astype(np.uint8)  # byte k: dim k of both tokens
+            w = value_unit_swizzle(r, d)
+            for u in range(8):
+                dst = r * d + (u ^ w) * unit
+                out[n, dst:dst + unit] = pair[u * unit:(u + 1) * unit]
+        out[n, BLOCK_TOKENS * (d // 2):] = full_scales[n * BLOCK_TOKENS:(n + 1) * BLOCK_TOKENS].astype("<u2").view(np.uint8)
+    return out
+
+
+def unpack_value_blocks(blocks, n_tokens: int, d: int):
+    """Inverse of pack_value_blocks: codes uint8 [n_tokens, d], scales uint16 [n_tokens]."""
+    blocks = np.asarray(blocks, dtype=np.uint8)
+    nb = blocks.shape[0]
+    unit = d // 8
+    codes = np.empty((nb * BLOCK_TOKENS, d), dtype=np.uint8)
+    for n in range(nb):
+        for r in range(BLOCK_TOKENS // 2):
+            w = value_unit_swizzle(r, d)
+            pair = np.empty(d, dtype=np.uint8)
+            for u in range(8):
+                src = r * d + (u ^ w) * unit
+                pair[u * unit:(u + 1) * unit] = blocks[n, src:src + unit]
+            codes[n * BLOCK_TOKENS + 2 * r] = pair & 0x0F
+            codes[n * BLOCK_TOKENS + 2 * r + 1] = pair >> 4
+    sc = np.ascontiguousarray(blocks[:, BLOCK_TOKENS * (d // 2):]).view("<u2").reshape(-1)
+    return codes[:n_tokens], sc[:n_tokens].astype(np.uint16)
 
 
 def unpack_blocks(blocks, n_tokens: int, d: int):

@@ -42,6 +42,8 @@ def test_abi_version_and_status_strings(akv):
     assert akv.abi_version() == 1
     assert akv.status_string(0) == "ok"
     assert akv.status_string(-9) == "page id out of bounds"
+    assert akv.status_string(-10) == "kernel launch configuration defect"
+    assert akv.error_word_status(akv.AKV_EFLAG_INTERNAL | akv.AKV_EFLAG_TIMEOUT) == akv.AKV_ERR_INTERNAL
     assert akv.error_word_status(0) == 0
     assert akv.error_word_status(akv.AKV_EFLAG_RANGE) == akv.AKV_ERR_RANGE
     assert akv.error_word_status(akv.AKV_EFLAG_RANGE | akv.AKV_EFLAG_BOUNDS) == akv.AKV_ERR_BOUNDS

@@ -120,9 +120,9 @@ def test_encode_bit_exact(akv, wlmod, cuda, d, paged):
                         synth.f32_to_bf16_bits(np.full((1, d), 3.0, np.float32))])  # exact ties possible
     kb, vb, err = _encode_case(akv, wlmod, cuda, x, d, paged)
     assert err == 0
-    for blocks, xs in ((kb, x), (vb, x[::-1])):
+    for blocks, xs, pack in ((kb, x, ora.pack_blocks), (vb, x[::-1], ora.pack_value_blocks)):
         enc = ora.encode(xs)
-        want = ora.pack_blocks(enc.codes, enc.scale_bits)
+        want = pack(enc.codes, enc.scale_bits)
         assert np.array_equal(blocks, want)
 
 
@@ -138,6 +138,8 @@ def test_encode_refusals_flag_and_zero_encode(akv, wlmod, cuda):
     enc = ora.encode(x)
     assert enc.nonfinite[3] and enc.nonfinite[9] and enc.overflow[20]
     assert np.array_equal(kb, ora.pack_blocks(enc.codes, enc.scale_bits))
+    ev = ora.encode(x[::-1])
+    assert np.array_equal(vb, ora.pack_value_blocks(ev.codes, ev.scale_bits))
 
 
 # ----------------------------------------------------------------------------------
@@ -237,7 +239,7 @@ def _oracle_hybrid(wl, w, b, heads=None):
         ev = ora.encode(vv[h, :Tc])
         kh[h] = ora.dequantize(ek.codes, ek.scale_bits)
         vh[h] = ora.dequantize(ev.codes, ev.scale_bits)
-        codes.append((ora.pack_blocks(ek.codes, ek.scale_bits), ora.pack_blocks(ev.codes, ev.scale_bits)))
+        codes.append((ora.pack_blocks(ek.codes, ek.scale_bits), ora.pack_value_blocks(ev.codes, ev.scale_bits)))
     tiers = [(kh, vh), (f64(kk[:, Tc:]), f64(vv[:, Tc:]))]
     return ora.decode_sequence(f64(w.q_bits[b]), tiers, wl.scale, wl.split_tokens), codes
 
@@ -280,7 +282,7 @@ def test_hybrid_full_size_sampled(akv, wlmod, cuda, variant):
             ek = ora.encode(w.k_bits[b, h, :Tc])
             ev = ora.encode(w.v_bits[b, h, :Tc])
             assert np.array_equal(kc[b, h], ora.pack_blocks(ek.codes, ek.scale_bits))
-            assert np.array_equal(vc[b, h], ora.pack_blocks(ev.codes, ev.scale_bits))
+            assert np.array_equal(vc[b, h], ora.pack_value_blocks(ev.codes, ev.scale_bits))
             kh = ora.dequantize(ek.codes, ek.scale_bits)[None]
             vh = ora.dequantize(ev.codes, ev.scale_bits)[None]
             qh = f64(w.q_bits[b, h * G:(h + 1) * G])

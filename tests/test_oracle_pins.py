@@ -243,6 +243,45 @@ def test_pack_and_block_layout_by_hand():
     assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
 
 
+def test_value_block_layout_by_hand():
+    # codes chosen so every (token, dim) is recognisable: code = (7 * t + 3 * dim) mod 16
+    def codes_for(n, d):
+        t = np.arange(n)[:, None]
+        dim = np.arange(d)[None, :]
+        return ((7 * t + 3 * dim) % 16).astype(np.uint8)
+    # d = 64: pair row r at byte 64 r, units of 8 bytes, unit u at position u ^ w(r)
+    d = 64
+    c = codes_for(17, d)
+    sc = (np.arange(17, dtype=np.uint16) + 1) * 0x0102
+    vb = ora.pack_value_blocks(c, sc)
+    assert vb.shape == (2, 544)
+    # tokens 0, 1 dim 0: pair row 0, w = 0 -> byte 0
+    assert vb[0, 0] == c[0, 0] | c[1, 0] << 4 == 0x70
+    # tokens 4, 5 dim 0: pair row 2, w = 4 -> unit 0 at position 4 -> byte 128 + 32 = 160
+    assert vb[0, 160] == c[4, 0] | c[5, 0] << 4 == 0x3C
+    # tokens 6, 7 dim 9: pair row 3, w = 4 -> unit 1 at position 5 -> byte 192 + 40 + 1 = 233
+    assert vb[0, 233] == c[6, 9] | c[7, 9] << 4 == 0xC5
+    # tokens 2, 3 dim 9: pair row 1, w = 0 -> byte 64 + 9 = 73
+    assert vb[0, 73] == c[2, 9] | c[3, 9] << 4 == 0x09
+    # scales as for keys: token 5 at 16 * 32 + 10, little-endian
+    assert vb[0, 522:524].tolist() == [0x0C, 0x06]
+    # token 16 heads block 1 (paired with a padding token of code 7), the rest is padding
+    assert vb[1, 0] == c[16, 0] | 7 << 4
+    assert np.all(vb[1, 64:512] == 0x77) and np.all(vb[1, 514:] == 0)
+    c2, s2 = ora.unpack_value_blocks(vb, 17, d)
+    assert np.array_equal(c2, c) and np.array_equal(s2, sc)
+    # d = 128: units of 16 bytes, w(r) = 2 (r mod 4)
+    d = 128
+    c = codes_for(16, d)
+    vb = ora.pack_value_blocks(c, np.zeros(16, np.uint16))
+    # tokens 2, 3 dim 17: pair row 1, w = 2 -> unit 1 at position 3 -> byte 128 + 48 + 1 = 177
+    assert vb[0, 177] == c[2, 17] | c[3, 17] << 4 == 0x81
+    # tokens 14, 15 dim 127: pair row 7, w = 6 -> unit 7 at position 1 -> byte 896 + 16 + 15 = 927
+    assert vb[0, 927] == c[14, 127] | c[15, 127] << 4 == 0x6F
+    c2, _ = ora.unpack_value_blocks(vb, 16, d)
+    assert np.array_equal(c2, c)
+
+
 def test_dequantize_reproduces_table():
     # d = 64 and s = 8 = sqrt(64): y_i = s * c[code_i] / sqrt(d) = c[code_i] exactly
     codes = np.tile(np.arange(16, dtype=np.uint8), 4)[None, :]
