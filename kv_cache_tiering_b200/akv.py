@@ -184,6 +184,23 @@ class Tier:
                         self.stride_token, lens.ctypes.data, None if slots is None else slots.ctypes.data)
 
 
+class TierArray:
+    """A tier list marshalled once for repeated calls.  Holds its own references to the
+    tiers' host arrays, so later changes to the Tier objects do not affect it; build a new
+    one when the tiers change."""
+
+    def __init__(self, tiers):
+        self.tiers = list(tiers)
+        cs = [t.c() for t in self.tiers]
+        self._keep = [t._keep for t in self.tiers]
+        self.arr = (AkvTierC * max(1, len(cs)))(*cs)
+        self.n = len(cs)
+
+
+def _tier_array(tiers) -> TierArray:
+    return tiers if isinstance(tiers, TierArray) else TierArray(tiers)
+
+
 def abi_version() -> int:
     return lib.akv_abi_version()
 
@@ -225,12 +242,10 @@ def akv_encode_history(src: Tier, dst: Tier, B: int, Hkv: int, d: int, err_word=
 def akv_decode_attend(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int,
                       o_part, lse_part, n_slots: int, variant: int = AKV_VARIANT_AUTO, err_word=None,
                       stream=None) -> None:
-    cs = [t.c() for t in tiers]
-    arr = (AkvTierC * max(1, len(cs)))(*cs)
-    _check(lib.akv_decode_attend(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens,
+    ta = _tier_array(tiers)
+    _check(lib.akv_decode_attend(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens,
                                  _ptr(o_part), _ptr(lse_part), int(n_slots), variant, _ptr(err_word),
                                  _stream(stream)))
-    del cs
 
 
 def akv_merge_lse(o_part, lse_part, n_slots: int, seq_slot_base, seq_n_slots, B: int, Hq: int, d: int, o, lse,
@@ -242,31 +257,26 @@ def akv_merge_lse(o_part, lse_part, n_slots: int, seq_slot_base, seq_n_slots, B:
 
 
 def akv_decode_workspace_size(B: int, Hq: int, Hkv: int, d: int, tiers, split_tokens: int) -> int:
-    cs = [t.c() for t in tiers]
-    arr = (AkvTierC * max(1, len(cs)))(*cs)
+    ta = _tier_array(tiers)
     n = ctypes.c_size_t(0)
-    _check(lib.akv_decode_workspace_size(B, Hq, Hkv, d, arr, len(cs), split_tokens, ctypes.byref(n)))
+    _check(lib.akv_decode_workspace_size(B, Hq, Hkv, d, ta.arr, ta.n, split_tokens, ctypes.byref(n)))
     return n.value
 
 
 def akv_decode(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int, workspace,
                workspace_bytes: int, o, lse, variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
-    cs = [t.c() for t in tiers]
-    arr = (AkvTierC * max(1, len(cs)))(*cs)
-    _check(lib.akv_decode(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens, _ptr(workspace),
+    ta = _tier_array(tiers)
+    _check(lib.akv_decode(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens, _ptr(workspace),
                           int(workspace_bytes), _ptr(o), _ptr(lse), variant, _ptr(err_word), _stream(stream)))
-    del cs
 
 
 def akv_decode_static(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int, o, lse,
                       variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
     """akv_decode on the library's own fixed scratch, for callers that cannot allocate
     device memory when they decode; see include/akv.h for its limits."""
-    cs = [t.c() for t in tiers]
-    arr = (AkvTierC * max(1, len(cs)))(*cs)
-    _check(lib.akv_decode_static(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), arr, len(cs), split_tokens, _ptr(o),
+    ta = _tier_array(tiers)
+    _check(lib.akv_decode_static(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens, _ptr(o),
                                  _ptr(lse), variant, _ptr(err_word), _stream(stream)))
-    del cs
 
 
 class Stager:

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/akv.h"
 
 namespace akv {
@@ -143,6 +145,45 @@ __device__ __forceinline__ const uint8_t* codes_block(const TierDev& t, const ui
     blk = (int64_t)b * t.s_seq + (int64_t)h * t.s_head + (int64_t)(tok >> 4) * t.s_tok;
   }
   return base + blk * BB;
+}
+
+// ------------------------------------------------------------------------------------
+// per-device launch set-up, done once
+// ------------------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+
+// Raise `Kernel`'s dynamic shared-memory limit on the current device to at least `bytes`.
+// The runtime keeps the attribute, so only the first launch that needs more pays the call.
+template <auto Kernel>
+inline cudaError_t ensure_smem(int bytes) {
+  static std::atomic<int> have[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && have[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+    int cur = have[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !have[dev].compare_exchange_weak(cur, bytes)) {
+    }
+  }
+  return e;
+}
+
+// Streaming multiprocessors of the current device (queried once per device).
+inline int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 0 ? n : 1;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // ------------------------------------------------------------------------------------

@@ -1073,20 +1073,13 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   cp_async_wait<0>();
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 1;
-}
-
 template <int D, int G>
 cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s) {
   constexpr int NW = 8;
   constexpr int NST = G <= 4 ? 3 : 2;
   using C = Bf16Cfg<D, G, NW, NST>;
   auto k = attend_bf16_mma<D, G, NW, NST>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  cudaError_t e = ensure_smem<attend_bf16_mma<D, G, NW, NST>>((int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   const int grid = n_items < sms ? n_items : sms;
@@ -1100,7 +1093,7 @@ cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
   constexpr int NST = 4;
   using C = CodesCfg<D, G, NWARP, NST>;
   auto k = attend_codes_mma<D, G, NWARP, NST>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  cudaError_t e = ensure_smem<attend_codes_mma<D, G, NWARP, NST>>((int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   const int grid = n_items < sms ? n_items : sms;

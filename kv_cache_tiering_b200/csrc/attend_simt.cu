@@ -454,13 +454,13 @@ cudaError_t launch_simt_dg(const AttendParams& p, int kind, int n_items, cudaStr
   if (kind == AKV_TIER_BF16) {
     const size_t sm = (size_t)(p.split_tokens * G + G * D) * sizeof(float);
     auto k = attend_bf16_simt<D, G>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = ensure_smem<attend_bf16_simt<D, G>>((int)sm);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, sm, s>>>(p);
   } else {
     const size_t sm = (size_t)(p.split_tokens * G + 2 * G * D) * sizeof(float);
     auto k = attend_codes_simt<D, G>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = ensure_smem<attend_codes_simt<D, G>>((int)sm);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, sm, s>>>(p);
   }

@@ -37,21 +37,24 @@ class DecodeStep:
         self.o = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
         self.lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
-        self.ws_bytes = akv.akv_decode_workspace_size(B, Hq, Hkv, d, tiers, split_tokens)
+        # the tier list marshalled once for every call of the step
+        self.tiers_c = akv.TierArray(tiers)
+        self.tier_c = [akv.TierArray([t]) for t in tiers]
+        self.ws_bytes = akv.akv_decode_workspace_size(B, Hq, Hkv, d, self.tiers_c, split_tokens)
         self.workspace = torch.zeros(max(256, self.ws_bytes), dtype=torch.uint8, device=device)
 
     def decode(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
         """The whole step in one call (split attention with the merge fused in)."""
-        akv.akv_decode(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens, self.workspace,
+        akv.akv_decode(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers_c, self.split_tokens, self.workspace,
                        self.ws_bytes, self.o, self.lse, variant, self.err, stream)
 
     def attend(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
-        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers, self.split_tokens,
+        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers_c, self.split_tokens,
                               self.o_part, self.lse_part, self.n_slots, variant, self.err, stream)
 
     def attend_tier(self, i: int, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
         """Tier i alone: the same launch ``attend`` makes for it, into the same slots."""
-        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, [self.tiers[i]], self.split_tokens,
+        akv.akv_decode_attend(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tier_c[i], self.split_tokens,
                               self.o_part, self.lse_part, self.n_slots, variant, self.err, stream)
 
     def merge(self, stream=None):

@@ -138,3 +138,20 @@ def test_stager_host_refusals(akv):
         st.use(5)
     assert e.value.status == akv.AKV_ERR_INVALID
     st.destroy()
+
+
+def test_tier_array_keeps_its_host_arrays(akv):
+    """A marshalled tier list stays valid after its Tier objects are marshalled again
+    (each marshalling makes fresh host int32 copies)."""
+    import ctypes
+    t = akv.Tier(akv.AKV_TIER_BF16, 0x1000, 0x2000, lens=[5, 0, 17], slot_base=[0, 1, 1],
+                 stride_seq=64, stride_head=0, stride_token=8)
+    ta = akv.TierArray([t])
+    for _ in range(3):
+        t.c()  # replaces the Tier's own kept arrays
+    import gc
+    gc.collect()
+    lens = ctypes.cast(ta.arr[0].lens, ctypes.POINTER(ctypes.c_int32))
+    slots = ctypes.cast(ta.arr[0].slot_base, ctypes.POINTER(ctypes.c_int32))
+    assert [lens[i] for i in range(3)] == [5, 0, 17] and [slots[i] for i in range(3)] == [0, 1, 1]
+    assert ta.n == 1 and akv.TierArray(ta.tiers).n == 1
