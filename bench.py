@@ -39,7 +39,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny", "staged"])
+    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny", "staged", "staged-hybrid"])
     ap.add_argument("--layers", type=int, default=None, help="staged workload: layers (default 16)")
     ap.add_argument("--variant", default="auto", choices=["auto", "simt", "mma"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -176,6 +176,8 @@ def describe(name, wl, w):
         "tiny": "tiny exact decode: batch 1, 1 q / 1 KV head, d 64, 256 BF16 tokens, 4 splits of 64",
         "hybrid": "hybrid tier: batch 4, 32 q / 8 KV heads, d 128, 32768 tokens (newest 2048 BF16, 30720 4-bit codes)",
         "ragged": "ragged paged hybrid: batch 64, lengths U[1024, 65536], 16-token pages, newest 1024 BF16",
+        "staged-hybrid": "staged 128k hybrid history: batch 1, 16 layers, 32 q / 8 KV heads, d 128, newest 2048 "
+                         "tokens BF16 on the device, 129024 compact in pinned host memory, 4096-token chunks",
         "staged": "staged 128k history: batch 1, 16 layers, 32 q / 8 KV heads, d 128, 131072 BF16 tokens per layer "
                   "in pinned host memory, 4096-token chunks through a 2-buffer device region, one token appended "
                   "per step",
@@ -189,6 +191,10 @@ def describe(name, wl, w):
 # ----------------------------------------------------------------------------------
 # reference arm: the float64 CPU oracle
 # ----------------------------------------------------------------------------------
+
+
+def _codes(enc):
+    return enc.codes, enc.scale_bits
 
 
 def oracle_sequence_fn(name, wl, seed_rank=0):
@@ -222,6 +228,20 @@ def oracle_sequence_fn(name, wl, seed_rank=0):
             ora.decode_sequence(f64(q[b, h * G:(h + 1) * G]), tiers, wl.scale, wl.split_tokens)
             return T / wl.Hkv
         return fn, wl.B * wl.Hkv, "one (sequence, KV head) with its 4 query heads per unit, encode included"
+    if name == "staged-hybrid":
+        n, W = 16384, wl.extra["window"]  # one layer's decode over a 16384-token sample per unit
+        gen = synth.stream(wl.seed, "oracle-sample-hybrid")
+
+        def fn(i):
+            k = synth.normal_bf16(gen, (wl.Hkv, n, wl.d))
+            v = synth.normal_bf16(gen, (wl.Hkv, n, wl.d))
+            q = synth.normal_bf16(gen, (wl.Hq, wl.d))
+            kh = np.stack([ora.dequantize(*_codes(ora.encode(k[h, :n - W]))) for h in range(wl.Hkv)])
+            vh = np.stack([ora.dequantize(*_codes(ora.encode(v[h, :n - W]))) for h in range(wl.Hkv)])
+            ora.decode_sequence(f64(q), [(kh, vh), (f64(k[:, n - W:]), f64(v[:, n - W:]))], wl.scale,
+                                wl.split_tokens)
+            return n
+        return fn, 4, "one layer's decode over a 16384-token sample (14336 compact, encode included) per unit"
     if name == "staged":
         n = 16384  # tokens of one layer per unit (a bounded sample of the 131072-token layer)
         gen = synth.stream(wl.seed, "oracle-sample")
@@ -507,12 +527,25 @@ def run_staged(args):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
-    base = synth.WORKLOADS["staged"]
+    hybrid = args.workload == "staged-hybrid"
+    base = synth.WORKLOADS[args.workload]
     wl = synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.d, base.split_tokens, seed=base.seed + rank,
                         extra=dict(base.extra))
     layers = args.layers or wl.extra["layers"]
     n_steps = max(3, args.warmup) + args.steps
-    st = workloads.StagedDecode(wl, dev, layers=layers, max_steps=n_steps + 1)
+    if hybrid:
+        st = workloads.StagedHybridDecode(wl, dev, layers=layers, T=wl.extra["T"], W=wl.extra["window"],
+                                          chunk=wl.extra["chunk"], max_steps=n_steps + 1)
+    else:
+        st = workloads.StagedDecode(wl, dev, layers=layers, max_steps=n_steps + 1)
+    o_host = torch.empty(st.o.shape, dtype=torch.float32).pin_memory()
+    lse_host = torch.empty(st.lse.shape, dtype=torch.float32).pin_memory()
+
+    def one_step(i):
+        st.step(*inputs[i], variant)
+        with torch.cuda.stream(st.compute_stream):  # the step's result, read back every step
+            o_host.copy_(st.o, non_blocking=True)
+            lse_host.copy_(st.lse, non_blocking=True)
     variant = {"auto": akv.AKV_VARIANT_AUTO, "simt": akv.AKV_VARIANT_SIMT, "mma": akv.AKV_VARIANT_MMA}[args.variant]
     inputs = [st.inputs(i) for i in range(n_steps)]
     # pinned host -> device copy bandwidth of this machine (the PCIe roofline)
@@ -530,7 +563,7 @@ def run_staged(args):
     sampler = ClockSampler(local)
     sampler.start()
     for i in range(max(3, args.warmup)):
-        st.step(*inputs[i], variant)
+        one_step(i)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -538,7 +571,7 @@ def run_staged(args):
     tw0 = time.monotonic()
     t0 = time.perf_counter()
     for i in range(max(3, args.warmup), n_steps):
-        st.step(*inputs[i], variant)
+        one_step(i)
     torch.cuda.synchronize()
     dt = time.perf_counter() - t0
     tw1 = time.monotonic()
@@ -557,9 +590,13 @@ def run_staged(args):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "staged 128k history: batch 1, %d layers, 32 q / 8 KV heads, d 128, "
-                                       "131072 BF16 tokens per layer in pinned host memory, 4096-token chunks "
-                                       "through a 2-buffer device region, one token appended per step" % layers,
+                "config": {"workload": ("staged 128k hybrid history: batch 1, %d layers, 32 q / 8 KV heads, d 128, "
+                                        "131072 tokens per layer: newest 2048 BF16 on the device, 129024 as 4-bit "
+                                        "codes in pinned host memory, 4096-token chunks through a 2-buffer device "
+                                        "region, one token appended per step" if hybrid else
+                                        "staged 128k history: batch 1, %d layers, 32 q / 8 KV heads, d 128, "
+                                        "131072 BF16 tokens per layer in pinned host memory, 4096-token chunks "
+                                        "through a 2-buffer device region, one token appended per step") % layers,
                            "timing": "host wall clock, timing-disabled fences", "parallelism":
                            f"independent replicas x{world}", "variant": args.variant},
                 "roofline": {"bound": "pcie", "achieved": pcie, "peak": pcie_peak, "unit": "GB/s",
@@ -567,9 +604,17 @@ def run_staged(args):
                              "peak_source": "pinned 256 MiB host-to-device copy measured in this run"},
                 "pcie_h2d_gbs": pcie, "h2d_bytes_per_step": h2d // args.steps,
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d // args.steps,
-                        "d2h_bytes_per_step": layers * st.row_bytes},
-                "gpu_launches": args.steps * layers * (-(-(wl.extra["T"] + 1) // st.chunk) + 1),
+                        "d2h_bytes_per_step": (0 if hybrid else layers * st.row_bytes)
+                        + 4 * (o_host.numel() + lse_host.numel())},
+                # attention launches per layer (one per staged chunk, plus the window for the
+                # hybrid) and the merge
+                "gpu_launches": args.steps * layers * (
+                    (-(-st.Tc // st.chunk) + 2) if hybrid else (-(-(wl.extra["T"] + 1) // st.chunk) + 1)),
                 "clocks": sampler.summary(tw0, tw1), "device_error_word": err}
+        if world == 1 and not args.no_cpu_baseline:
+            cv, units, desc, odt = time_oracle(args.workload, wl)
+            line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                    "sample": f"{units} units ({desc}), {odt:.1f} s"}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -581,7 +626,7 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload == "staged":
+    if args.workload in ("staged", "staged-hybrid"):
         return run_staged(args)
     return run_ours(args)
 

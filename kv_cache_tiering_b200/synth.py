@@ -16,6 +16,8 @@ library is measured on):
            compact; K, V ~ N(0,1)
   staged   batch 1, 16 layers, 32 / 8 heads, d 128, 131072 tokens per layer in pinned
            host memory, token-major, 4096-token chunks, one new token per step
+  staged-hybrid  the staged shape with the newest 2048 tokens per layer BF16 on the device
+           and the older 129024 compact in pinned host memory, staged in 4096-token chunks
   ragged   batch 64, lengths uniform in [1024, 65536], 16-token pages with a seeded
            random page permutation, newest 1024 exact, K ~ Student-t(3), V, q ~ N(0,1)
 """
@@ -80,6 +82,8 @@ WORKLOADS = {
                        extra={"T": 32768, "window": 2048}),
     "staged": Workload("staged", B=1, Hq=32, Hkv=8, d=128, split_tokens=512,
                        extra={"T": 131072, "layers": 16, "chunk": 4096, "buffers": 2}),
+    "staged-hybrid": Workload("staged-hybrid", B=1, Hq=32, Hkv=8, d=128, split_tokens=512,
+                              extra={"T": 131072, "layers": 16, "chunk": 4096, "buffers": 2, "window": 2048}),
     "ragged": Workload("ragged", B=64, Hq=32, Hkv=8, d=128, split_tokens=512,
                        extra={"min_len": 1024, "max_len": 65536, "window": 1024, "nu": 3.0}),
 }

@@ -362,3 +362,126 @@ class StagedDecode:
     def close(self):
         if not self.resident:
             self.stager.destroy()
+
+
+class StagedHybridDecode:
+    """The hybrid tier with its compact part staged from the host.
+
+    Per layer, tokens [0, Tc) live as compact blocks in pinned host memory, Tc = T - W, and
+    tokens [Tc, T + steps) stay BF16 on the device (the exact window, which the appended
+    tokens join).  Host layout of a layer: block rows [Tc/16][K | V][Hkv][block bytes] -- a
+    row holds the 16-token key blocks of every head, then the value blocks -- so a run of
+    consecutive tokens is one contiguous span, about a quarter of its BF16 size.
+
+    A decode step, per layer: the new token's row is appended to the window; every chunk of
+    the compact part is staged through the ring (akv_stage_chunk on the copy stream) and
+    attended as a CODES4 tier into its own split slots; the window is attended from device
+    memory; the partials are merged.  ``resident=True`` keeps the same compact rows in device
+    memory and issues the same attend calls (the bit-identity comparison).  The compact
+    codes are written by the library's encoder from a seeded BF16 history."""
+
+    def __init__(self, wl: synth.Workload, device, layers: int, T: int, W: int, chunk: int, max_steps: int = 8,
+                 n_buffers: int = 2, resident: bool = False, source: str = "torch"):
+        assert chunk % wl.split_tokens == 0 and chunk % 16 == 0 and 0 < W <= T
+        self.wl, self.device, self.resident = wl, device, resident
+        self.L, self.T, self.W, self.chunk = layers, T, W, chunk
+        H, d = wl.Hkv, wl.d
+        self.Tc = T - W
+        self.bb = akv.codes4_block_bytes(d)
+        self.crow = 2 * H * self.bb                  # bytes of one 16-token block row
+        self.nrows = -(-self.Tc // 16)
+        self.wrow = 2 * H * d * 2                    # bytes of one BF16 window row
+        self.wcap = W + max_steps
+        self.host, self.win = [], []
+        self.k_bits, self.v_bits = [], []            # host copies of the BF16 history (source="host")
+        for layer in range(layers):
+            if source == "host":
+                kk, vv = synth.history_token_major(wl, layer, T)     # [T, Hkv, d]
+                self.k_bits.append(kk)
+                self.v_bits.append(vv)
+                k_dev = to_dev_bits(np.ascontiguousarray(kk.transpose(1, 0, 2)), device)
+                v_dev = to_dev_bits(np.ascontiguousarray(vv.transpose(1, 0, 2)), device)
+            else:
+                g = synth.torch_generator(wl.seed, wl.name, "staged-hybrid", layer, device=device)
+                k_dev = synth.torch_normal_bf16(g, (H, T, d), device)
+                v_dev = synth.torch_normal_bf16(g, (H, T, d), device)
+            codes = torch.empty(max(1, self.nrows) * self.crow, dtype=torch.uint8, device=device)
+            if self.Tc > 0:
+                src = akv.Tier(akv.AKV_TIER_BF16, k_dev, v_dev, lens=[self.Tc], stride_seq=0, stride_head=T * d,
+                               stride_token=d)
+                dst = akv.Tier(akv.AKV_TIER_CODES4, codes, codes.data_ptr() + H * self.bb, lens=[self.Tc],
+                               stride_seq=0, stride_head=1, stride_token=2 * H)
+                enc_err = torch.zeros(1, dtype=torch.int32, device=device)
+                akv.akv_encode_history(src, dst, 1, H, d, enc_err)
+            win = torch.zeros((self.wcap, 2, H, d), dtype=torch.int16, device=device)
+            win[:W, 0] = k_dev[:, self.Tc:T].transpose(0, 1)
+            win[:W, 1] = v_dev[:, self.Tc:T].transpose(0, 1)
+            self.win.append(win)
+            self.host.append(codes if resident else codes.cpu().pin_memory())
+            del k_dev, v_dev
+        torch.cuda.synchronize(device)
+        self.copy_stream = torch.cuda.Stream(device)
+        self.compute_stream = torch.cuda.Stream(device)
+        if not resident:
+            rows = -(-min(chunk, max(16, self.Tc)) // 16)          # block rows of the largest chunk
+            per_buf = -(-(rows * self.crow) // 256) * 256
+            self.region = torch.empty(n_buffers * per_buf, dtype=torch.uint8, device=device)
+            self.stager = akv.Stager(self.region, self.region.numel(), n_buffers)
+        self.n_cslots = -(-self.Tc // wl.split_tokens)
+        n_slots = self.n_cslots + -(-self.wcap // wl.split_tokens)
+        self.o_part = torch.empty((n_slots, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty((n_slots, wl.Hq), dtype=torch.float32, device=device)
+        self.o = torch.empty((layers, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse = torch.empty((layers, wl.Hq), dtype=torch.float32, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.steps_done = 0
+        self.h2d_bytes = 0
+
+    def inputs(self, step: int):
+        """Device q [L][Hq][d] and new rows [L][2][Hkv][d] of decode step ``step``."""
+        q = np.stack([synth.queries(self.wl, layer=l, step=step, B=1)[0] for l in range(self.L)])
+        new = np.stack([np.stack(synth.new_token(self.wl, l, step)) for l in range(self.L)])
+        return to_dev_bits(q, self.device), to_dev_bits(new, self.device)
+
+    def step(self, q, new_rows, variant=akv.AKV_VARIANT_AUTO, timeout_ms: int = -1):
+        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device)."""
+        wl, H, d = self.wl, self.wl.Hkv, self.wl.d
+        cs = self.compute_stream
+        nw = self.W + self.steps_done + 1           # window tokens including the appended one
+        per_chunk = self.chunk // wl.split_tokens
+        n_wsplit = -(-nw // wl.split_tokens)
+        n_chunks = -(-self.Tc // self.chunk)
+        for layer in range(self.L):
+            win = self.win[layer]
+            with torch.cuda.stream(cs):
+                win[nw - 1].copy_(new_rows[layer])
+            for c in range(n_chunks):
+                tok0 = c * self.chunk
+                ntc = min(self.chunk, self.Tc - tok0)
+                row0, nrow = tok0 // 16, -(-ntc // 16)
+                buf = None
+                if self.resident:
+                    base = self.host[layer].data_ptr() + row0 * self.crow
+                else:
+                    buf, base = self.stager.stage_chunk(self.host[layer].data_ptr() + row0 * self.crow,
+                                                        nrow * self.crow, self.copy_stream, timeout_ms)
+                    self.h2d_bytes += nrow * self.crow
+                    self.stager.use(buf, cs)
+                tier = akv.Tier(akv.AKV_TIER_CODES4, base, base + H * self.bb, lens=[ntc], slot_base=[c * per_chunk],
+                                stride_seq=0, stride_head=1, stride_token=2 * H)
+                akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
+                                      self.lse_part, self.o_part.shape[0], variant, self.err, cs)
+                if buf is not None:
+                    self.stager.release(buf, cs)
+            wb = win.data_ptr()
+            tier = akv.Tier(akv.AKV_TIER_BF16, wb, wb + H * d * 2, lens=[nw], slot_base=[self.n_cslots],
+                            stride_seq=0, stride_head=d, stride_token=2 * H * d)
+            akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
+                                  self.lse_part, self.o_part.shape[0], variant, self.err, cs)
+            akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [self.n_cslots + n_wsplit], 1,
+                              wl.Hq, d, self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
+        self.steps_done += 1
+
+    def close(self):
+        if not self.resident:
+            self.stager.destroy()

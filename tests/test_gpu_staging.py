@@ -59,6 +59,48 @@ def test_staged_equals_resident_bitwise_and_oracle(mods, cuda, T):
     staged.close()
 
 
+@pytest.mark.parametrize("T,W", [(9003, 1000), (4700, 4096)])
+def test_staged_hybrid_equals_resident_bitwise_and_oracle(mods, cuda, T, W):
+    """Compact history staged from pinned host memory (a partial last block and a partial
+    last chunk when T - W = 8003; a single short chunk when T - W = 604), window resident."""
+    import torch
+    akv, workloads = mods
+    wl = synth.Workload("staged-hybrid-small", B=1, Hq=32, Hkv=8, d=128, split_tokens=512, extra={})
+    kw = dict(layers=2, T=T, W=W, chunk=4096, max_steps=3, source="host")
+    staged = workloads.StagedHybridDecode(wl, cuda, **kw)
+    resident = workloads.StagedHybridDecode(wl, cuda, resident=True, **kw)
+    Tc = T - W
+    assert staged.h2d_bytes == 0
+    for step in range(2):
+        q, new = staged.inputs(step)
+        staged.step(q, new)
+        resident.step(q, new)
+        torch.cuda.synchronize()
+        assert torch.equal(staged.o, resident.o) and torch.equal(staged.lse, resident.lse)
+        assert int(staged.err.item()) == 0
+    # every step stages the whole compact part: ceil(Tc / 16) block rows of 2 x 8 x 1056 bytes per layer
+    assert staged.h2d_bytes == 2 * 2 * (-(-Tc // 16)) * 2 * 8 * 1056
+    # oracle: layer 1 after step 1 -- compact tokens [0, Tc) encoded, window [Tc, T) + 2 appended
+    layer = 1
+    k, v = staged.k_bits[layer], staged.v_bits[layer]                     # [T, Hkv, d]
+    kh = np.zeros((8, Tc, 128))
+    vh = np.zeros((8, Tc, 128))
+    for h in range(8):
+        ek, ev = ora.encode(k[:Tc, h]), ora.encode(v[:Tc, h])
+        kh[h] = ora.dequantize(ek.codes, ek.scale_bits)
+        vh[h] = ora.dequantize(ev.codes, ev.scale_bits)
+    k_new = np.stack([synth.new_token(wl, layer, s)[0] for s in range(2)])
+    v_new = np.stack([synth.new_token(wl, layer, s)[1] for s in range(2)])
+    kwin = np.concatenate([k[Tc:], k_new]).transpose(1, 0, 2)
+    vwin = np.concatenate([v[Tc:], v_new]).transpose(1, 0, 2)
+    tiers = [(kh, vh), (ora.bf16_bits_to_f64(kwin), ora.bf16_bits_to_f64(vwin))]
+    q1 = synth.queries(wl, layer=layer, step=1, B=1)[0]
+    _, _, (o_ref, l_ref) = ora.decode_sequence(ora.bf16_bits_to_f64(q1), tiers, wl.scale, wl.split_tokens)
+    assert np.max(np.abs(staged.o[layer].cpu().numpy() - o_ref)) <= 2e-3
+    assert np.max(np.abs(staged.lse[layer].cpu().numpy() - l_ref)) <= 1e-3
+    staged.close()
+
+
 def test_stager_refuses_pageable_memory(mods, cuda):
     import torch
     akv, _ = mods
