@@ -39,7 +39,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny", "staged", "staged-hybrid"])
+    ap.add_argument("--workload", default="exact", choices=["exact", "hybrid", "ragged", "tiny", "staged", "staged-hybrid", "aging"])
     ap.add_argument("--layers", type=int, default=None, help="staged workload: layers (default 16)")
     ap.add_argument("--variant", default="auto", choices=["auto", "simt", "mma"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -622,12 +622,82 @@ def run_staged(args):
     return 0
 
 
+def run_aging(args):
+    """Live hybrid decode with window aging on the hybrid shape: every step appends a token
+    per sequence; every 16 steps each window hands its oldest page to the compact tier.
+    Timed with CUDA events on the step's stream, whole steps and the parts."""
+    import torch
+    from kv_cache_tiering_b200 import akv, synth, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    base = synth.WORKLOADS["hybrid"]
+    wl = synth.Workload("aging", base.B, base.Hq, base.Hkv, base.d, base.split_tokens, seed=base.seed + rank,
+                        extra=dict(base.extra))
+    T, W = wl.extra["T"], wl.extra["window"]
+    n_warm = max(3, args.warmup)
+    n_steps = n_warm + args.steps
+    st = workloads.AgingHybrid(wl, dev, [T] * wl.B, W, max_steps=n_steps + 1, source="torch")
+    variant = {"auto": akv.AKV_VARIANT_AUTO, "simt": akv.AKV_VARIANT_SIMT, "mma": akv.AKV_VARIANT_MMA}[args.variant]
+    inputs = [st.inputs(i) for i in range(n_steps)]
+    stream = torch.cuda.current_stream()
+    for i in range(n_warm):
+        st.step(*inputs[i], variant, stream)
+    torch.cuda.synchronize()
+    aged0, tok = st.aged_blocks, 0
+    st.encode_events = []
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_warm, n_steps):
+        tok += int(st.c.sum() + st.win.sum()) + wl.B
+        st.step(*inputs[i], variant, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        ms = max_over_ranks(ms, dist, dev)
+    aged = st.aged_blocks - aged0
+    enc_us = [a.elapsed_time(b) * 1e3 for a, b in st.encode_events]
+    value = tok * world / (ms * 1e-3)
+    err = int(st.err.item())
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "window aging on the hybrid shape: batch 4, 32 q / 8 KV heads, d 128, "
+                                       "32768 tokens, newest 2048-2063 BF16 in 16-token ring pages, the rest 4-bit "
+                                       "code pages; one token appended per step, full window pages encoded into "
+                                       "the compact tier", "parallelism": f"independent replicas x{world}",
+                           "variant": args.variant, "timing": "CUDA events around whole steps"},
+                "aged_blocks_in_timed_steps": int(aged) * wl.Hkv, "aging_events": len(enc_us),
+                "aging_encode_us_avg": sum(enc_us) / max(1, len(enc_us)),
+                "e2e": None, "gpu_launches": args.steps * 3 + int(aged > 0) * (aged // wl.B),
+                "device_error_word": err}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload in ("staged", "staged-hybrid"):
         return run_staged(args)
+    if args.workload == "aging":
+        return run_aging(args)
     return run_ours(args)
 
 

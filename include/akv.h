@@ -140,6 +140,24 @@ typedef struct akv_tier {
 } akv_tier;
 
 /* ------------------------------------------------------------------------------------
+ * akv_append_tokens -- write each sequence's new token into a BF16 tier.
+ *
+ * A decode step first appends the new token's key and value to the history, then attends
+ * ("Context beyond VRAM", "What I built": the step appends the new K/V and attends).  For
+ * every sequence b < B with pos[b] >= 0, the key row new_k[b][h][:] and value row
+ * new_v[b][h][:] of every KV head h go to token pos[b] of `tier`, addressed exactly as
+ * attention reads it (contiguous strides, or the page table for paged tiers).
+ * tier: kind BF16, paged or contiguous; its lens and slot_base are not used; its k and v
+ * rows at the given positions are WRITTEN.  new_k, new_v: device bf16 [B][Hkv][d], 16-byte
+ * aligned.  pos: host int32 [B], the tier-relative token index (negative: skip b).  A paged
+ * position whose page id is outside the pool sets AKV_EFLAG_BOUNDS in *err_word (device, may
+ * be NULL) and writes nothing for that sequence.  Validation errors launch nothing; B = 0
+ * or all positions negative is a no-op.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_append_tokens(const akv_tier* tier, const int32_t* pos, int B, int Hkv, int d, const void* new_k,
+                             const void* new_v, int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * akv_encode_history -- rotate, quantise and pack BF16 history into the compact tier.
  *
  * For every sequence b < B, KV head h < Hkv and token t < dst->lens[b], the BF16 key and

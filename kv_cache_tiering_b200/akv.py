@@ -104,6 +104,8 @@ _sig("akv_decode_workspace_size", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctyp
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t))
 _sig("akv_decode", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, _p, _p)
+_sig("akv_append_tokens", ctypes.c_int, ctypes.POINTER(AkvTierC), _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
+     _p, _p, _p)
 _sig("akv_decode_static", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, _p, ctypes.c_int, _p, _p)
 _sig("akv_stager_create", ctypes.c_int, _p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_p))
@@ -232,6 +234,14 @@ def plan_slots(tier_lens, split_tokens: int):
     _check(lib.akv_plan_slots(B, len(lens), lp, split_tokens, bp, seq_base.ctypes.data, seq_n.ctypes.data,
                               ctypes.byref(n)))
     return bases, seq_base, seq_n, n.value
+
+
+def akv_append_tokens(tier: Tier, pos, B: int, Hkv: int, d: int, new_k, new_v, err_word=None, stream=None) -> None:
+    """Write row b of new_k / new_v ([B][Hkv][d] bf16, device) to token pos[b] of a BF16 tier."""
+    t = tier.c()
+    p = _host_i32(pos)
+    _check(lib.akv_append_tokens(ctypes.byref(t), p.ctypes.data, B, Hkv, d, _ptr(new_k), _ptr(new_v), _ptr(err_word),
+                                 _stream(stream)))
 
 
 def akv_encode_history(src: Tier, dst: Tier, B: int, Hkv: int, d: int, err_word=None, stream=None) -> None:

@@ -72,6 +72,16 @@ struct EncodeParams {
   SeqTable seq;          // items are 16-token blocks
 };
 
+struct AppendParams {
+  TierDev tier;          // BF16 tier whose rows are written
+  const uint16_t* new_k;  // [B][Hkv][D] bf16 (whole call)
+  const uint16_t* new_v;
+  int32_t* err;
+  int32_t Hkv;
+  int32_t b0;            // global index of the launch's first sequence
+  int32_t pos[kMaxSeqPerLaunch];
+};
+
 struct MergeParams {
   const float* o_part;
   const float* lse_part;
@@ -191,6 +201,7 @@ inline int sm_count() {
 // ------------------------------------------------------------------------------------
 
 cudaError_t launch_encode(const EncodeParams& p, int d, int n_items, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, int d, int n_seq, cudaStream_t s);
 cudaError_t launch_attend_simt(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
 cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
 // Fill p.tmk / p.tmv for a BF16 tier of B sequences (tokens [0, max_len)): 4-D maps

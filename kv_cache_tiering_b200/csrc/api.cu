@@ -256,6 +256,49 @@ akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, i
   return ok();
 }
 
+akv_status akv_append_tokens(const akv_tier* tier, const int32_t* pos, int B, int Hkv, int d, const void* new_k,
+                             const void* new_v, int32_t* err_word, akv_stream_t stream) {
+  if (B < 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "B must be >= 0 and Hkv > 0");
+  if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (Hkv > 65535) return fail(AKV_ERR_UNSUPPORTED, "Hkv %d too large", Hkv);
+  if (!tier) return fail(AKV_ERR_INVALID, "tier is null");
+  if (tier->kind != AKV_TIER_BF16) return fail(AKV_ERR_INVALID, "tokens are appended to a BF16 tier");
+  if (B == 0) return ok();
+  if (!pos) return fail(AKV_ERR_INVALID, "pos is null");
+  if (err_word && !aligned(err_word, 4)) return fail(AKV_ERR_INVALID, "err_word must be 4-byte aligned");
+  // validate the tier as if it held tokens [0, pos[b]] of every sequence
+  std::vector<int32_t> lens(B);
+  bool any = false;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] == INT32_MAX) return fail(AKV_ERR_INVALID, "pos[%d] too large", b);
+    lens[b] = pos[b] < 0 ? 0 : pos[b] + 1;
+    any |= pos[b] >= 0;
+  }
+  if (!any) return ok();
+  if (!new_k || !new_v || !aligned(new_k, 16) || !aligned(new_v, 16))
+    return fail(AKV_ERR_INVALID, "new_k and new_v must be 16-byte aligned device pointers");
+  akv_tier view = *tier;
+  view.lens = lens.data();
+  view.slot_base = nullptr;
+  akv_status s;
+  if ((s = check_tier(&view, 0, B, d, 16, false, 0, AKV_TIER_BF16)) != AKV_OK) return s;
+  akv::AppendParams p;
+  p.tier = tier_dev(&view);
+  p.new_k = static_cast<const uint16_t*>(new_k);
+  p.new_v = static_cast<const uint16_t*>(new_v);
+  p.err = err_word;
+  p.Hkv = Hkv;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+    const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+    p.b0 = b0;
+    for (int i = 0; i < n; ++i) p.pos[i] = pos[b0 + i];
+    cudaError_t e = akv::launch_append(p, d, n, st);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  return ok();
+}
+
 akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, int Hkv, int d, int32_t* err_word,
                               akv_stream_t stream) {
   if (B < 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "B must be >= 0 and Hkv > 0");

@@ -485,3 +485,164 @@ class StagedHybridDecode:
     def close(self):
         if not self.resident:
             self.stager.destroy()
+
+
+class AgingHybrid:
+    """A live hybrid batch whose exact window ages into the compact tier during decode.
+
+    Sequence b starts with c_b = 16 floor((L_b - W) / 16) compact tokens and L_b - c_b in
+    [W, W + 16) exact ones.  The exact window is a ring of R = W/16 + 2 pages of 16 BF16
+    tokens per sequence (pool [B R, Hkv, 16, d]); the compact history is a growing list of
+    code pages drawn from a seeded permutation of the code pool ([P, Hkv] blocks).  A decode
+    step appends each sequence's new token to its window; a window that reaches W + 16 tokens
+    has its oldest page encoded into the sequence's next code page (one akv_encode_history
+    call over every aging sequence) and that ring page leaves the window.  Then both tiers
+    are attended and merged.  Page tables live on the device; only entries that change are
+    written."""
+
+    def __init__(self, wl: synth.Workload, device, lens, W: int, max_steps: int, key_dist: str = "normal",
+                 source: str = "host"):
+        lens = np.asarray(lens, np.int64)
+        assert W % 16 == 0 and W > 0 and np.all(lens >= W)
+        H, d = wl.Hkv, wl.d
+        self.wl, self.device, self.B, self.W = wl, device, len(lens), W
+        self.bb = akv.codes4_block_bytes(d)
+        self.c = ((lens - W) // 16 * 16).astype(np.int64)       # compact tokens
+        self.win = (lens - self.c).astype(np.int64)              # exact tokens, in [W, W + 16)
+        self.R = W // 16 + 2
+        self.ring0 = np.zeros(self.B, np.int64)                  # ring page of the window's first page
+        cap = self.c // 16 + max_steps // 16 + 2
+        self.n_cp = int(cap.sum())
+        perm = synth.page_permutation(wl, "aging-codes", self.n_cp)
+        offs = np.concatenate([[0], np.cumsum(cap)])
+        self.owned = [perm[offs[b]:offs[b + 1]] for b in range(self.B)]
+        self.cp_table_np = np.full((self.B, int(cap.max())), -1, np.int32)
+        for b in range(self.B):
+            n = int(self.c[b] // 16)
+            self.cp_table_np[b, :n] = self.owned[b][:n]
+        self.ex_table_np = np.array([[b * self.R + j for j in range(self.R)] for b in range(self.B)], np.int32)
+        self.ex_k = torch.zeros((self.B * self.R, H, 16, d), dtype=torch.int16, device=device)
+        self.ex_v = torch.zeros_like(self.ex_k)
+        self.cp_k = torch.zeros((self.n_cp, H, self.bb), dtype=torch.uint8, device=device)
+        self.cp_v = torch.zeros_like(self.cp_k)
+        self.cp_table = torch.from_numpy(self.cp_table_np).to(device)
+        self.ex_table = torch.from_numpy(self.ex_table_np).to(device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.k_hist, self.v_hist = [], []                        # host BF16 history (source="host")
+        for b in range(self.B):
+            L, c = int(lens[b]), int(self.c[b])
+            if source == "host":
+                k, v = synth.history_head_major(wl, b, L, key_dist=key_dist)
+                self.k_hist.append(k)
+                self.v_hist.append(v)
+                kd, vd = to_dev_bits(k, device), to_dev_bits(v, device)
+            else:
+                g = synth.torch_generator(wl.seed, wl.name, "aging", b, device=device)
+                kd = synth.torch_student_t3_bf16(g, (H, L, d), device) if key_dist == "student_t" \
+                    else synth.torch_normal_bf16(g, (H, L, d), device)
+                vd = synth.torch_normal_bf16(g, (H, L, d), device)
+            if c > 0:
+                src = akv.Tier(akv.AKV_TIER_BF16, kd, vd, lens=[c], stride_seq=0, stride_head=L * d, stride_token=d)
+                dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True,
+                               page_table=self.cp_table[b:b + 1], page_table_stride=self.cp_table_np.shape[1],
+                               n_pages=self.n_cp, stride_seq=H, stride_head=1)
+                akv.akv_encode_history(src, dst, 1, H, d, self.err)
+            w = L - c
+            pages = -(-w // 16)
+            ek = torch.zeros((H, pages * 16, d), dtype=torch.int16, device=device)
+            ev = torch.zeros_like(ek)
+            ek[:, :w] = kd[:, c:]
+            ev[:, :w] = vd[:, c:]
+            self.ex_k[b * self.R:b * self.R + pages] = ek.view(H, pages, 16, d).permute(1, 0, 2, 3)
+            self.ex_v[b * self.R:b * self.R + pages] = ev.view(H, pages, 16, d).permute(1, 0, 2, 3)
+        torch.cuda.synchronize(device)
+        max_slots = int(sum(-(-(int(l) + max_steps) // wl.split_tokens) + 2 for l in lens))
+        self.o_part = torch.empty((max_slots, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty((max_slots, wl.Hq), dtype=torch.float32, device=device)
+        self.o = torch.empty((self.B, wl.Hq, d), dtype=torch.float32, device=device)
+        self.lse = torch.empty((self.B, wl.Hq), dtype=torch.float32, device=device)
+        self.q = to_dev_bits(synth.queries(wl, B=self.B), device)
+        self._cp_host = torch.empty(self.cp_table_np.shape, dtype=torch.int32).pin_memory()
+        self._ex_host = torch.empty(self.ex_table_np.shape, dtype=torch.int32).pin_memory()
+        self._enc_host = torch.empty((self.B, 2), dtype=torch.int32).pin_memory()
+        self._enc_dev = torch.empty((self.B, 2), dtype=torch.int32, device=device)
+        self._tables_done = torch.cuda.Event()
+        self._tables_done.record(torch.cuda.current_stream(device))
+        self.steps_done = 0
+        self.aged_blocks = 0
+        self.encode_events = None  # a list: every aging encode is bracketed by timing events
+
+    def inputs(self, step: int):
+        """Device q [B][Hq][d] and new K, V rows [B][Hkv][d] of decode step ``step``."""
+        wl = self.wl
+        q = synth.queries(wl, step=step + 1, B=self.B)
+        kn = np.stack([synth.new_token(wl, 0, step, b)[0] for b in range(self.B)])
+        vn = np.stack([synth.new_token(wl, 0, step, b)[1] for b in range(self.B)])
+        return to_dev_bits(q, self.device), to_dev_bits(kn, self.device), to_dev_bits(vn, self.device)
+
+    def _exact_tier(self, lens=None, slot_base=None):
+        H, d = self.wl.Hkv, self.wl.d
+        return akv.Tier(akv.AKV_TIER_BF16, self.ex_k, self.ex_v, lens=self.win if lens is None else lens,
+                        slot_base=slot_base, paged=True, page_table=self.ex_table, page_table_stride=self.R,
+                        n_pages=self.B * self.R, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
+
+    def _ex_row(self, b: int) -> np.ndarray:
+        return np.array([b * self.R + (self.ring0[b] + j) % self.R for j in range(self.R)], np.int32)
+
+    def step(self, q, k_new, v_new, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        """Append one token per sequence, age full window pages, attend both tiers, merge."""
+        wl, H, d, B = self.wl, self.wl.Hkv, self.wl.d, self.B
+        dev = self.device
+        # 1. append: token win[b] of the window, through the window's page table
+        akv.akv_append_tokens(self._exact_tier(), self.win.astype(np.int32), B, H, d, k_new, v_new, self.err, stream)
+        self.win += 1
+        # 2. age: a window of W + 16 tokens hands its oldest page to the compact tier
+        aging = [b for b in range(B) if self.win[b] >= self.W + 16]
+        if aging:
+            n = len(aging)
+            self._tables_done.synchronize()   # the pinned buffers' previous uploads have finished
+            enc = self._enc_host[:n]
+            for i, b in enumerate(aging):
+                enc[i, 0] = b * self.R + self.ring0[b]                  # oldest window page
+                enc[i, 1] = int(self.owned[b][self.c[b] // 16])         # the next code page
+                self.cp_table_np[b, int(self.c[b] // 16)] = enc[i, 1]
+                self.c[b] += 16
+                self.ring0[b] = (self.ring0[b] + 1) % self.R
+                self.win[b] -= 16
+                self.ex_table_np[b] = self._ex_row(b)
+            self._cp_host.copy_(torch.from_numpy(self.cp_table_np))
+            self._ex_host.copy_(torch.from_numpy(self.ex_table_np))
+            cur = torch.cuda.current_stream(dev) if stream is None else stream
+            with torch.cuda.stream(cur):
+                self._enc_dev[:n].copy_(enc, non_blocking=True)
+                ptr = self._enc_dev.data_ptr()
+                # column 0 of the page lists addresses the source pages, column 1 the destination
+                src = akv.Tier(akv.AKV_TIER_BF16, self.ex_k, self.ex_v, lens=[16] * n, paged=True, page_table=ptr,
+                               page_table_stride=2, n_pages=B * self.R, stride_seq=H * 16 * d, stride_head=16 * d,
+                               stride_token=d)
+                dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[16] * n, paged=True,
+                               page_table=ptr + 4, page_table_stride=2, n_pages=self.n_cp, stride_seq=H,
+                               stride_head=1)
+                if self.encode_events is not None:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(cur)
+                akv.akv_encode_history(src, dst, n, H, d, self.err, cur)
+                if self.encode_events is not None:
+                    e1.record(cur)
+                    self.encode_events.append((e0, e1))
+                self.cp_table.copy_(self._cp_host, non_blocking=True)
+                self.ex_table.copy_(self._ex_host, non_blocking=True)
+                self._tables_done.record(cur)
+            self.aged_blocks += n
+        # 3. attend both tiers into their planned slots, then merge
+        cp_len, ex_len = self.c.astype(np.int32), self.win.astype(np.int32)
+        bases, seq_base, seq_n, n_slots = akv.plan_slots([cp_len, ex_len], wl.split_tokens)
+        codes = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=cp_len, slot_base=bases[0], paged=True,
+                         page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1], n_pages=self.n_cp,
+                         stride_seq=H, stride_head=1)
+        exact = self._exact_tier(ex_len, bases[1])
+        akv.akv_decode_attend(q, B, wl.Hq, H, d, wl.scale, [codes, exact], wl.split_tokens, self.o_part,
+                              self.lse_part, n_slots, variant, self.err, stream)
+        akv.akv_merge_lse(self.o_part, self.lse_part, n_slots, seq_base, seq_n, B, wl.Hq, d, self.o, self.lse,
+                          stream)
+        self.steps_done += 1

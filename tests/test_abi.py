@@ -155,3 +155,20 @@ def test_tier_array_keeps_its_host_arrays(akv):
     slots = ctypes.cast(ta.arr[0].slot_base, ctypes.POINTER(ctypes.c_int32))
     assert [lens[i] for i in range(3)] == [5, 0, 17] and [slots[i] for i in range(3)] == [0, 1, 1]
     assert ta.n == 1 and akv.TierArray(ta.tiers).n == 1
+
+
+def test_append_tokens_refusals(akv):
+    import ctypes
+    t = akv.Tier(akv.AKV_TIER_CODES4, 0x1000, 0x2000, lens=[0])
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_append_tokens(t, [0], 1, 8, 128, 0x3000, 0x4000)
+    assert e.value.status == akv.AKV_ERR_INVALID
+    t = akv.Tier(akv.AKV_TIER_BF16, 0x1000, 0x2000, lens=[0], stride_seq=1024, stride_head=128, stride_token=8)
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_append_tokens(t, [3], 1, 8, 96, 0x3000, 0x4000)
+    assert e.value.status == akv.AKV_ERR_UNSUPPORTED
+    with pytest.raises(akv.AkvError) as e:
+        akv.akv_append_tokens(t, [3], 1, 8, 128, 0x3008, 0x4000)  # misaligned rows
+    assert e.value.status == akv.AKV_ERR_INVALID
+    akv.akv_append_tokens(t, [-1, -5], 2, 8, 128, 0x3000, 0x4000)  # nothing to write: no launch
+    assert akv.lib.akv_append_tokens(ctypes.byref(t.c()), None, 1, 8, 128, None, None, None, None) == akv.AKV_ERR_INVALID
