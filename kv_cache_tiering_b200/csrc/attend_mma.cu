@@ -716,9 +716,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     if (threadIdx.x == 0) flag_error(p.err, AKV_EFLAG_INTERNAL);
     return;
   }
-  // word i of this warp's scratch: word i % 32 of the upper half of its table row i / 32
+  // word i of this warp's scratch: in the upper half of its table row r = i / 32, at word
+  // (i % 32) ^ 4 (r % 8) -- the 16-byte units of a row are XOR-swizzled by the row, so the
+  // query-fragment reads and the rotation reads are conflict-free and the output writes
+  // at most 2-way
   const uint32_t scr_s = lut_s + (uint32_t)(warp * C::SCR_ROWS) * 256u + 128u;
-  auto scr = [&](int i) -> uint32_t { return scr_s + ((uint32_t)(i >> 5) << 8) + ((uint32_t)(i & 31) << 2); };
+  auto scr = [&](int i) -> uint32_t {
+    const uint32_t r = (uint32_t)i >> 5;
+    return scr_s + (r << 8) + ((((uint32_t)i & 31u) ^ ((r & 7u) << 2)) << 2);
+  };
 
   // this warp's item range: an equal share of all items, in item order; warps are numbered
   // warp-major across CTAs so a partly filled grid still spreads its busy warps over every SM
