@@ -267,6 +267,33 @@ akv_status akv_decode_static(const void* q, int B, int Hq, int Hkv, int d, float
                              int variant, int32_t* err_word, akv_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * Context checkpoints -- suspend a context to a file and resume it without recomputation
+ * ("Context beyond VRAM", "What I built": a checkpointed context lifecycle).  A context is
+ * whatever host spans its owner names (the pinned history of every layer, compact code
+ * rows, ...) plus n_meta uint64 values that describe them (layer count, lengths, steps).
+ *
+ * File layout (little-endian): the 8 bytes "AKVCKPT1", uint32 version (1), uint32 n_meta,
+ * uint32 n_spans, uint32 0, n_meta uint64 values, then per span uint64 byte count and
+ * uint32 CRC-32 (IEEE 802.3, reflected polynomial 0xEDB88320) with uint32 0, then the span
+ * bytes in order.
+ *
+ * akv_checkpoint_write: spans[i] are host pointers (pinned or pageable) of span_bytes[i]
+ * bytes.  The file is written to `path` plus ".tmp" and renamed onto `path` once complete,
+ * so a failed write never leaves a partial file under `path`.  I/O failures return
+ * AKV_ERR_INVALID with the system's message.  Synchronous; the caller orders it after the
+ * device work that produced the spans.
+ * akv_checkpoint_info: reads the counts, the meta values (up to *n_meta) and the span
+ * sizes (up to *n_spans); on return *n_meta and *n_spans hold the file's counts.
+ * akv_checkpoint_read: reads every span into caller buffers whose sizes must equal the
+ * recorded ones.  A file whose magic, version, counts, sizes or CRC-32 do not match is
+ * refused with AKV_ERR_INVALID (the buffers then hold unspecified bytes).
+ * ------------------------------------------------------------------------------------ */
+akv_status akv_checkpoint_write(const char* path, const uint64_t* meta, int n_meta, const void* const* spans,
+                                const uint64_t* span_bytes, int n_spans);
+akv_status akv_checkpoint_info(const char* path, uint64_t* meta, int* n_meta, uint64_t* span_bytes, int* n_spans);
+akv_status akv_checkpoint_read(const char* path, void* const* spans, const uint64_t* span_bytes, int n_spans);
+
+/* ------------------------------------------------------------------------------------
  * akv_plan_slots -- host helper: the standard slot layout.
  *
  * Sequence-major: sequence b owns a contiguous run of slots holding tier 0's splits,

@@ -106,6 +106,12 @@ _sig("akv_decode", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, c
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, _p, _p)
 _sig("akv_append_tokens", ctypes.c_int, ctypes.POINTER(AkvTierC), _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
      _p, _p, _p)
+_sig("akv_checkpoint_write", ctypes.c_int, ctypes.c_char_p, ctypes.POINTER(ctypes.c_uint64), ctypes.c_int,
+     ctypes.POINTER(_p), ctypes.POINTER(ctypes.c_uint64), ctypes.c_int)
+_sig("akv_checkpoint_info", ctypes.c_int, ctypes.c_char_p, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int),
+     ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int))
+_sig("akv_checkpoint_read", ctypes.c_int, ctypes.c_char_p, ctypes.POINTER(_p), ctypes.POINTER(ctypes.c_uint64),
+     ctypes.c_int)
 _sig("akv_decode_static", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, _p, ctypes.c_int, _p, _p)
 _sig("akv_stager_create", ctypes.c_int, _p, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_p))
@@ -287,6 +293,32 @@ def akv_decode_static(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float
     ta = _tier_array(tiers)
     _check(lib.akv_decode_static(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens, _ptr(o),
                                  _ptr(lse), variant, _ptr(err_word), _stream(stream)))
+
+
+def checkpoint_write(path: str, meta, spans) -> None:
+    """Write a context checkpoint: `meta` uint64 values, `spans` (host address, bytes) pairs."""
+    meta = list(meta)
+    m = (ctypes.c_uint64 * max(1, len(meta)))(*meta)
+    ptrs = (_p * max(1, len(spans)))(*[_ptr(a) for a, _ in spans])
+    sizes = (ctypes.c_uint64 * max(1, len(spans)))(*[int(n) for _, n in spans])
+    _check(lib.akv_checkpoint_write(os.fsencode(path), m, len(meta), ptrs, sizes, len(spans)))
+
+
+def checkpoint_info(path: str):
+    """(meta values, span sizes) of a checkpoint file."""
+    nm, ns = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.akv_checkpoint_info(os.fsencode(path), None, ctypes.byref(nm), None, ctypes.byref(ns)))
+    m = (ctypes.c_uint64 * max(1, nm.value))()
+    z = (ctypes.c_uint64 * max(1, ns.value))()
+    _check(lib.akv_checkpoint_info(os.fsencode(path), m, ctypes.byref(nm), z, ctypes.byref(ns)))
+    return [int(m[i]) for i in range(nm.value)], [int(z[i]) for i in range(ns.value)]
+
+
+def checkpoint_read(path: str, spans) -> None:
+    """Read a checkpoint's spans into (host address, bytes) buffers of the recorded sizes."""
+    ptrs = (_p * max(1, len(spans)))(*[_ptr(a) for a, _ in spans])
+    sizes = (ctypes.c_uint64 * max(1, len(spans)))(*[int(n) for _, n in spans])
+    _check(lib.akv_checkpoint_read(os.fsencode(path), ptrs, sizes, len(spans)))
 
 
 class Stager:

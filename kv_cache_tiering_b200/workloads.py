@@ -303,6 +303,7 @@ class StagedDecode:
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
         self.steps_done = 0
         self.h2d_bytes = 0
+        self._wb_events = [None] * self.L  # per layer: the last write-back of an appended row
 
     def inputs(self, step: int):
         """Device q [L][Hq][d] and new rows [L][2][Hkv][d] of decode step ``step``."""
@@ -320,6 +321,8 @@ class StagedDecode:
         n_split = -(-n_tok // wl.split_tokens)
         per_chunk = self.chunk // wl.split_tokens
         rb = self.row_bytes
+        # the step's inputs come from the caller's stream
+        cs.wait_stream(torch.cuda.current_stream(self.device))
         for layer in range(self.L):
             new_row = new_rows[layer].reshape(-1).view(torch.uint8)
             for c in range(n_chunks):
@@ -333,6 +336,9 @@ class StagedDecode:
                     off = tok0 * rb
                 else:
                     src = self.host[layer].data_ptr() + tok0 * rb
+                    if tok0 <= pos - 1 < tok0 + self.chunk and self._wb_events[layer] is not None:
+                        # the previous step wrote row pos - 1 back to this chunk's host span
+                        self.copy_stream.wait_event(self._wb_events[layer])
                     buf, dev = self.stager.stage_chunk(src, have * rb, self.copy_stream, timeout_ms)
                     self.h2d_bytes += have * rb
                     self.stager.use(buf, cs)
@@ -353,11 +359,37 @@ class StagedDecode:
                         else:
                             self.stager.writeback(buf, (pos - tok0) * rb, self.host[layer].data_ptr() + pos * rb,
                                                   rb, cs)
+                            ev = torch.cuda.Event()
+                            ev.record(cs)
+                            self._wb_events[layer] = ev
                 if buf is not None:
                     self.stager.release(buf, cs)
             akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [n_split], 1, wl.Hq, d,
                               self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
+        torch.cuda.current_stream(self.device).wait_stream(cs)  # the results, for the caller's stream
         self.steps_done += 1
+
+    def suspend(self, path: str) -> None:
+        """Checkpoint the context: every layer's pinned history (the authoritative copy) and
+        the step count.  Device state is a working set rebuilt on resume."""
+        torch.cuda.synchronize(self.device)  # write-backs of the last step have landed
+        wl = self.wl
+        meta = [1, self.L, self.T, self.cap, self.chunk, self.steps_done, wl.Hkv, wl.d, wl.seed]
+        akv.checkpoint_write(path, meta, [(h.data_ptr(), h.numel() * h.element_size()) for h in self.host])
+
+    @classmethod
+    def resume(cls, path: str, wl: synth.Workload, device, n_buffers: int = 2, resident: bool = False):
+        """Rebuild a suspended context from its checkpoint, ready for its next step."""
+        meta, sizes = akv.checkpoint_info(path)
+        kind, L, T, cap, chunk, steps, hkv, d, _seed = meta
+        if kind != 1 or hkv != wl.Hkv or d != wl.d:
+            raise ValueError("checkpoint does not hold a staged BF16 context of this shape")
+        host = [torch.empty((cap, 2, hkv, d), dtype=torch.int16).pin_memory() for _ in range(L)]
+        akv.checkpoint_read(path, [(h.data_ptr(), n) for h, n in zip(host, sizes)])
+        st = cls(wl, device, layers=L, T=T, chunk=chunk, max_steps=cap - T, n_buffers=n_buffers, resident=resident,
+                 host_layers=host)
+        st.steps_done = steps
+        return st
 
     def close(self):
         if not self.resident:
@@ -451,6 +483,7 @@ class StagedHybridDecode:
         per_chunk = self.chunk // wl.split_tokens
         n_wsplit = -(-nw // wl.split_tokens)
         n_chunks = -(-self.Tc // self.chunk)
+        cs.wait_stream(torch.cuda.current_stream(self.device))  # the step's inputs
         for layer in range(self.L):
             win = self.win[layer]
             with torch.cuda.stream(cs):
@@ -480,6 +513,7 @@ class StagedHybridDecode:
                                   self.lse_part, self.o_part.shape[0], variant, self.err, cs)
             akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [self.n_cslots + n_wsplit], 1,
                               wl.Hq, d, self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
+        torch.cuda.current_stream(self.device).wait_stream(cs)  # the results, for the caller's stream
         self.steps_done += 1
 
     def close(self):

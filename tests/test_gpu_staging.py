@@ -101,6 +101,37 @@ def test_staged_hybrid_equals_resident_bitwise_and_oracle(mods, cuda, T, W):
     staged.close()
 
 
+def test_suspend_and_resume_continue_bit_identically(mods, cuda, tmp_path):
+    """A context suspended after two steps and resumed from its checkpoint produces the same
+    bits on its next steps as a run that never stopped."""
+    import torch
+    akv, workloads = mods
+    wl = _wl(5000)
+    path = str(tmp_path / "ctx.ckpt")
+    ref = workloads.StagedDecode(wl, cuda, max_steps=6)
+    run = workloads.StagedDecode(wl, cuda, max_steps=6)
+    for step in range(2):
+        ref.step(*ref.inputs(step))
+        run.step(*run.inputs(step))
+    run.suspend(path)
+    run.close()
+    del run
+    meta, sizes = akv.checkpoint_info(path)
+    assert meta[5] == 2 and len(sizes) == wl.extra["layers"]
+    res = workloads.StagedDecode.resume(path, wl, cuda)
+    assert res.steps_done == 2
+    for step in range(2, 4):
+        q, new = ref.inputs(step)
+        ref.step(q, new)
+        res.step(q, new)
+        torch.cuda.synchronize()
+        assert torch.equal(ref.o, res.o) and torch.equal(ref.lse, res.lse)
+    for layer in range(wl.extra["layers"]):
+        assert torch.equal(ref.host[layer], res.host[layer])
+    ref.close()
+    res.close()
+
+
 def test_stager_refuses_pageable_memory(mods, cuda):
     import torch
     akv, _ = mods
