@@ -44,6 +44,11 @@ Readings where the pages are silent (the plainest reading the rest supports):
     then the 16 scales as for keys.  (This is the order the tensor-core product reads.)
   * Dequantisation: y_i = s * c[code_i] / sqrt(d) in the rotated domain,
     x_hat = H y / sqrt(d) in the original domain.
+  * Rotation signs (the pages only name "Hadamard vs QR" trade-offs): an optional
+    randomised rotation flips the signs of the coordinates whose bits are set before the
+    transform, z = H (s . x), and the inverse applies them after, x_hat = s . (H y) / sqrt(d).
+    With no bits set both reduce to the plain transform.  H S is still orthogonal up to
+    the factor d, so the query is rotated the same way and dot products are preserved.
   * Softmax scale sigma is applied inside; LSE is the natural log of sum exp(scores);
     GQA head h reads KV head floor(h / G); an empty token range gives O = 0,
     LSE = -inf; splits of ``split_tokens`` tokens are aligned to the start of their
@@ -131,10 +136,22 @@ class Encoded:
     overflow: np.ndarray     # bool [n]: the norm rounds to binary16 infinity
 
 
-def encode(x_bits) -> Encoded:
+def sign_vector(sign_bits: int, d: int) -> np.ndarray:
+    """s_i = -1 where bit i of sign_bits is set, else +1 (float64 [d])."""
+    return np.array([-1.0 if (sign_bits >> i) & 1 else 1.0 for i in range(d)])
+
+
+def rotate(x, sign_bits: int = 0) -> np.ndarray:
+    """H (s . x), unnormalised, along the last axis."""
+    x = np.asarray(x, dtype=np.float64)
+    return fwht(x * sign_vector(sign_bits, x.shape[-1]))
+
+
+def encode(x_bits, sign_bits: int = 0) -> Encoded:
     """Rotate, scale and quantise BF16 vectors x_bits uint16 [n, d].
 
-    z = H x (unnormalised), s = binary16(||x||), code_i = #{j : z_i > s * b_j}.
+    z = H (s . x) (unnormalised; s = +1 everywhere when sign_bits = 0), s = binary16(||x||),
+    code_i = #{j : z_i > s * b_j}.
     A vector with a non-finite coordinate, or whose norm rounds to binary16 infinity,
     is refused: it is flagged and written as the zero-vector encoding (codes 7, scale 0).
     """
@@ -142,7 +159,7 @@ def encode(x_bits) -> Encoded:
     n, d = x.shape
     nonfinite = ~np.all(np.isfinite(x), axis=1)
     xs = np.where(np.isfinite(x), x, 0.0)
-    z = fwht(xs)
+    z = rotate(xs, sign_bits)
     s_bits = scale_f16_bits(xs)
     s = f16_bits_to_f64(s_bits)
     overflow = np.isinf(s)
@@ -267,10 +284,10 @@ def dequantize_rotated(codes, scale_bits) -> np.ndarray:
     return s[..., None] * c[codes] / math.sqrt(d)
 
 
-def dequantize(codes, scale_bits) -> np.ndarray:
-    """x_hat = H y / sqrt(d): the reconstructed vector in the original basis."""
+def dequantize(codes, scale_bits, sign_bits: int = 0) -> np.ndarray:
+    """x_hat = s . (H y) / sqrt(d): the reconstructed vector in the original basis."""
     y = dequantize_rotated(codes, scale_bits)
-    return fwht(y) / math.sqrt(y.shape[-1])
+    return fwht(y) / math.sqrt(y.shape[-1]) * sign_vector(sign_bits, y.shape[-1])
 
 
 # ----------------------------------------------------------------------------------

@@ -406,3 +406,32 @@ def test_decode_sequence_merge_equals_direct():
     partials, (mo, ml), (do, dl) = ora.decode_sequence(q, tiers, 0.2, 16)
     assert [p[0].shape[0] for p in partials] == [5, 3]
     assert np.allclose(mo, do, atol=1e-12) and np.allclose(ml, dl, atol=1e-12)
+
+
+def test_rotation_signs_by_hand_and_by_property():
+    # d = 2: H = [[1, 1], [1, -1]]; bit 1 set negates coordinate 1 before the transform
+    assert ora.rotate(np.array([3.0, 5.0]), 0b10).tolist() == [-2.0, 8.0]
+    assert ora.rotate(np.array([3.0, 5.0]), 0b01).tolist() == [2.0, -8.0]
+    assert ora.rotate(np.array([3.0, 5.0]), 0).tolist() == [8.0, -2.0]
+    d = 128
+    gen = np.random.default_rng(5)
+    bits = int(gen.integers(0, 2**62)) | (int(gen.integers(0, 2**62)) << 64)
+    x = _bf16(gen.standard_normal((6, d)))
+    # encoding with signs = encoding the sign-flipped input (bf16 sign flips are exact)
+    flip = np.array([(bits >> i) & 1 for i in range(d)], dtype=np.uint16) << 15
+    enc_s = ora.encode(x, bits)
+    enc_f = ora.encode(x ^ flip)
+    assert np.array_equal(enc_s.codes, enc_f.codes) and np.array_equal(enc_s.scale_bits, enc_f.scale_bits)
+    # (H S) (H S)^T = d I, so rotated queries keep dot products
+    M = np.stack([ora.rotate(e, bits) for e in np.eye(d)])
+    assert np.allclose(M @ M.T, d * np.eye(d), atol=0, rtol=0)
+    # the inverse applies the signs after the transform: the round trip stays within the
+    # quantiser's error, while the wrong order would not
+    xf = ora.bf16_bits_to_f64(x)
+    xh = ora.dequantize(enc_s.codes, enc_s.scale_bits, bits)
+    rel = np.sum((xh - xf) ** 2, axis=1) / np.sum(xf ** 2, axis=1)
+    assert np.all(rel < 0.02)
+    wrong = ora.fwht(ora.sign_vector(bits, d) * ora.dequantize_rotated(enc_s.codes, enc_s.scale_bits)) / np.sqrt(d)
+    assert np.all(np.sum((wrong - xf) ** 2, axis=1) / np.sum(xf ** 2, axis=1) > 0.5)
+    # no bits: the plain transform
+    assert np.array_equal(ora.encode(x, 0).codes, ora.encode(x).codes)
