@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define AKV_ABI_VERSION 1
+#define AKV_ABI_VERSION 2
 
 /* Opaque CUDA stream (cudaStream_t); 0 is the legacy default stream. */
 typedef struct CUstream_st* akv_stream_t;
@@ -123,6 +123,14 @@ enum { AKV_TIER_BF16 = 0, AKV_TIER_CODES4 = 1 };
  * slot_base[b] (host) is the partial-output slot of the tier's first split for sequence
  * b; split s (tokens [s*split_tokens, (s+1)*split_tokens) of the tier) goes to slot
  * slot_base[b] + s.  Splits are aligned to the start of the tier.
+ *
+ * rotation_signs (CODES4 only): bit i (word i / 32, bit i % 32) set negates coordinate i
+ * before the Walsh-Hadamard transform -- a randomised rotation z = H (s . x) of the
+ * compact form, read back as x = s . (H y) / d.  All zero is the plain transform.  The
+ * encoder and the attention kernels take the signs from the compact tier, so a tier must
+ * be read with the signs it was written with.  Bits at and above d are ignored.  (The
+ * pages name only the trade-off between Hadamard and QR rotations; this is the variant
+ * that keeps the fast transform.)
  */
 typedef struct akv_tier {
   int32_t kind;                  /* AKV_TIER_BF16 or AKV_TIER_CODES4 */
@@ -137,6 +145,7 @@ typedef struct akv_tier {
   int64_t stride_token;          /* see the addressing above; ignored for paged CODES4 */
   const int32_t* lens;           /* host [B] */
   const int32_t* slot_base;      /* host [B] */
+  uint32_t rotation_signs[4];    /* CODES4: coordinate sign flips before the rotation */
 } akv_tier;
 
 /* ------------------------------------------------------------------------------------

@@ -77,6 +77,7 @@ class AkvTierC(ctypes.Structure):
         ("stride_token", ctypes.c_int64),
         ("lens", _p),
         ("slot_base", _p),
+        ("rotation_signs", ctypes.c_uint32 * 4),
     ]
 
 
@@ -181,15 +182,17 @@ class Tier:
     page_table: object = None
     page_table_stride: int = 0
     n_pages: int = 0
+    rotation_signs: int = 0  # CODES4: bit i negates coordinate i before the rotation
     _keep: list = field(default_factory=list, repr=False)
 
     def c(self) -> AkvTierC:
         lens = _host_i32(self.lens)
         slots = _host_i32(self.slot_base) if self.slot_base is not None else None
         self._keep = [lens, slots]
+        signs = (ctypes.c_uint32 * 4)(*[(int(self.rotation_signs) >> (32 * i)) & 0xFFFFFFFF for i in range(4)])
         return AkvTierC(self.kind, 1 if self.paged else 0, _ptr(self.k), _ptr(self.v), _ptr(self.page_table),
                         self.page_table_stride, self.n_pages, self.stride_seq, self.stride_head,
-                        self.stride_token, lens.ctypes.data, None if slots is None else slots.ctypes.data)
+                        self.stride_token, lens.ctypes.data, None if slots is None else slots.ctypes.data, signs)
 
 
 class TierArray:

@@ -29,7 +29,13 @@ struct TierDev {
   int64_t n_pages;
   int64_t s_seq, s_head, s_tok;
   int32_t paged;
+  uint32_t signs[4];  // CODES4: coordinate i negated before the rotation when bit i is set
 };
+
+// +1 or -1: the rotation sign of coordinate i of a compact tier.
+__device__ __forceinline__ float coord_sign(const TierDev& t, int i) {
+  return ((t.signs[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f;
+}
 
 // Per-launch sequence table: work item i of the launch belongs to the sequence b with
 // item_base[b] <= i < item_base[b + 1]; b is local to the launch, b0 + b is global.

@@ -96,6 +96,7 @@ akv::TierDev tier_dev(const akv_tier* t) {
   td.s_head = t->stride_head;
   td.s_tok = t->stride_token;
   td.paged = t->paged;
+  for (int i = 0; i < 4; ++i) td.signs[i] = t->kind == AKV_TIER_CODES4 ? t->rotation_signs[i] : 0u;
   return td;
 }
 

@@ -878,9 +878,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int j = 0; j < P / 2; ++j) {
-          x[h][2 * j] = bf16lo(qw[h][j]);
-          x[h][2 * j + 1] = bf16hi(qw[h][j]);
+        for (int j = 0; j < P / 2; ++j) {  // the tier's rotation signs come first
+          x[h][2 * j] = bf16lo(qw[h][j]) * coord_sign(p.tier, P * lane + 2 * j);
+          x[h][2 * j + 1] = bf16hi(qw[h][j]) * coord_sign(p.tier, P * lane + 2 * j + 1);
         }
 #pragma unroll
       for (int h = 0; h < G; ++h) warp_fwht<P>(x[h]);
@@ -1056,6 +1056,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
       }
       warp_fwht<P>(x);
+#pragma unroll
+      for (int j = 0; j < P; ++j) x[j] *= coord_sign(p.tier, P * lane + j);  // undo the rotation signs
       float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
       if constexpr (P == 4) {
         *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);

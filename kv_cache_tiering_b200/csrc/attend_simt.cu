@@ -323,10 +323,10 @@ __global__ void __launch_bounds__(kThreads) attend_codes_simt(const __grid_const
     lut[i] = make_float2(half_bits_to_float(p.centroids[i & 15]), half_bits_to_float(p.centroids[i >> 4]));
   for (int i = threadIdx.x; i < G * D; i += kThreads) {
     const int h = i / D, dd = i % D;
-    qr[i] = bf16_to_float(p.q[((size_t)si.b * p.Hq + (size_t)si.kvh * G + h) * D + dd]);
+    qr[i] = bf16_to_float(p.q[((size_t)si.b * p.Hq + (size_t)si.kvh * G + h) * D + dd]) * coord_sign(p.tier, dd);
   }
   __syncthreads();
-  smem_fwht<D, G>(qr);  // qr = H q (unnormalised); ends with __syncthreads
+  smem_fwht<D, G>(qr);  // qr = H (s . q) (unnormalised); ends with __syncthreads
 
   // score_t (base 2) = scale_log2 * s_t / D * (H q) . c[codes_t]
   const float kfac = p.scale_log2 / (float)D;
@@ -435,12 +435,12 @@ __global__ void __launch_bounds__(kThreads) attend_codes_simt(const __grid_const
     }
     reduce_pv<D, G>(acc, red, dg, ph);
   }
-  // rotate back: O = H acc / (D * l)
+  // rotate back: O = s . (H acc) / (D * l)
   smem_fwht<D, G>(red);
   for (int i = threadIdx.x; i < G * D; i += kThreads) {
     const int h = i / D, dd = i % D;
     const int hq = si.kvh * G + h;
-    p.o_part[((size_t)si.slot * p.Hq + hq) * D + dd] = red[i] / ((float)D * sm_l[h]);
+    p.o_part[((size_t)si.slot * p.Hq + hq) * D + dd] = red[i] * coord_sign(p.tier, dd) / ((float)D * sm_l[h]);
   }
   if (threadIdx.x < G) {
     const int h = threadIdx.x;

@@ -25,7 +25,7 @@ namespace {
 // code_row, its binary16 scale to scale_slot.
 template <int D>
 __device__ __forceinline__ void encode_vector(const uint8_t* src_row, uint8_t* code_row, uint16_t* scale_slot,
-                                              bool valid, const double* bound, int32_t* err) {
+                                              bool valid, const double* bound, const uint32_t* signs, int32_t* err) {
   constexpr int P = D / 32;  // coordinates per lane: 4 (d = 128) or 2 (d = 64)
   const int lane = threadIdx.x & 31;
   double z[P];
@@ -59,6 +59,13 @@ __device__ __forceinline__ void encode_vector(const uint8_t* src_row, uint8_t* c
   }
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, m));
+
+  // the tier's rotation signs: coordinate i negated before the transform (exact)
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const int c = P * lane + i;
+    if ((signs[c >> 5] >> (c & 31)) & 1u) z[i] = -z[i];
+  }
 
   // in-lane butterflies (h < P)
 #pragma unroll
@@ -134,9 +141,9 @@ __global__ void __launch_bounds__(512) encode_kernel(const __grid_constant__ Enc
   // unit u of d/8 bytes at position u ^ w(r) -- the order the tensor-core product reads
   __shared__ __align__(16) uint8_t vrows[16 * ROWB];
   encode_vector<D>(ksrc, kblock + row * ROWB, reinterpret_cast<uint16_t*>(kblock + 16 * ROWB) + row, valid, bound,
-                   p.err);
+                   p.dst.signs, p.err);
   encode_vector<D>(vsrc, vrows + row * ROWB, reinterpret_cast<uint16_t*>(vblock + 16 * ROWB) + row, valid, bound,
-                   p.err);
+                   p.dst.signs, p.err);
   __syncthreads();
   // 8 pair rows of D bytes = 16 ROWB bytes; thread i writes 4 bytes of pair row i / (D/4)
   constexpr int US = D / 8;

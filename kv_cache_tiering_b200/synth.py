@@ -157,6 +157,12 @@ def scatter_pages(tokens_hd: np.ndarray, table_row: np.ndarray, pool: np.ndarray
         pool[table_row[j], :, : e - a, :] = tokens_hd[:, a:e, :]
 
 
+def rotation_sign_bits(seed: int, d: int, key: str = "signs") -> int:
+    """d random bits (bit i: coordinate i's sign flip) for a randomised rotation."""
+    bits = stream(seed, "rotation", key).integers(0, 2, size=d)
+    return int(sum(int(b) << i for i, b in enumerate(bits)))
+
+
 # ----------------------------------------------------------------------------------
 # device-side generators for full-size workloads (same distributions, BF16 rounding RNE)
 # ----------------------------------------------------------------------------------

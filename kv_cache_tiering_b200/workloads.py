@@ -107,11 +107,13 @@ class HybridResident:
     """Hybrid tiers of one batch: tokens [0, T - W) compact (contiguous code blocks
     [B, Hkv, (T - W)/16]), tokens [T - W, T) exact BF16 (a view of the head-major history)."""
 
-    def __init__(self, wl: synth.Workload, device, B: int | None = None, T: int | None = None, W: int | None = None):
+    def __init__(self, wl: synth.Workload, device, B: int | None = None, T: int | None = None, W: int | None = None,
+                 rotation_signs: int = 0):
         self.wl = wl
         B = wl.B if B is None else B
         T = wl.extra["T"] if T is None else T
         W = wl.extra["window"] if W is None else W
+        self.rotation_signs = rotation_signs
         self.B, self.T, self.W = B, T, W
         d, H = wl.d, wl.Hkv
         self.q_bits = synth.queries(wl, B=B)
@@ -133,7 +135,7 @@ class HybridResident:
         src = akv.Tier(akv.AKV_TIER_BF16, self.k, self.v, lens=np.full(B, Tc, np.int32),
                        stride_seq=H * T * d, stride_head=T * d, stride_token=d)
         self.codes_tier = akv.Tier(akv.AKV_TIER_CODES4, self.kc, self.vc, lens=np.full(B, Tc, np.int32),
-                                   stride_seq=H * nb, stride_head=nb, stride_token=1)
+                                   stride_seq=H * nb, stride_head=nb, stride_token=1, rotation_signs=rotation_signs)
         self.enc_err = torch.zeros(1, dtype=torch.int32, device=device)
         akv.akv_encode_history(src, self.codes_tier, B, H, d, self.enc_err)
         off = Tc * d * 2  # bytes: the window starts at token Tc of every (b, h) stream

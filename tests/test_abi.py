@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(akv):
 
 
 def test_abi_version_and_status_strings(akv):
-    assert akv.abi_version() == 1
+    assert akv.abi_version() == 2
     assert akv.status_string(0) == "ok"
     assert akv.status_string(-9) == "page id out of bounds"
     assert akv.status_string(-10) == "kernel launch configuration defect"

@@ -79,7 +79,7 @@ def check_merged(step, b, ref, hq_sel=None):
 # ----------------------------------------------------------------------------------
 
 
-def _encode_case(akv, wlmod, cuda, x_bits, d, paged):
+def _encode_case(akv, wlmod, cuda, x_bits, d, paged, signs=0):
     """Encode one (sequence, head) stream of n vectors [n, d] on the GPU; return its blocks."""
     import torch
     n = x_bits.shape[0]
@@ -95,11 +95,12 @@ def _encode_case(akv, wlmod, cuda, x_bits, d, paged):
         kc = torch.full((nb + 3, bb), 0xAB, dtype=torch.uint8, device=cuda)
         vc = torch.full((nb + 3, bb), 0xAB, dtype=torch.uint8, device=cuda)
         dst = akv.Tier(akv.AKV_TIER_CODES4, kc, vc, lens=[n], paged=True, page_table=table, page_table_stride=nb,
-                       n_pages=nb + 3, stride_seq=1, stride_head=0)
+                       n_pages=nb + 3, stride_seq=1, stride_head=0, rotation_signs=signs)
     else:
         kc = torch.full((nb, bb), 0xAB, dtype=torch.uint8, device=cuda)
         vc = torch.full((nb, bb), 0xAB, dtype=torch.uint8, device=cuda)
-        dst = akv.Tier(akv.AKV_TIER_CODES4, kc, vc, lens=[n], stride_seq=0, stride_head=0, stride_token=1)
+        dst = akv.Tier(akv.AKV_TIER_CODES4, kc, vc, lens=[n], stride_seq=0, stride_head=0, stride_token=1,
+                       rotation_signs=signs)
     akv.akv_encode_history(src, dst, 1, 1, d, err)
     torch.cuda.synchronize()
     kb, vb = kc.cpu().numpy(), vc.cpu().numpy()
@@ -124,6 +125,19 @@ def test_encode_bit_exact(akv, wlmod, cuda, d, paged):
         enc = ora.encode(xs)
         want = pack(enc.codes, enc.scale_bits)
         assert np.array_equal(blocks, want)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_encode_bit_exact_with_rotation_signs(akv, wlmod, cuda, d):
+    gen = synth.stream(0, "test-encode-signs", d)
+    x = np.concatenate([synth.normal_bf16(gen, (40, d)), synth.student_t_bf16(gen, (9, d), 3.0)])
+    bits = synth.rotation_sign_bits(0, d, "test-encode")
+    kb, vb, err = _encode_case(akv, wlmod, cuda, x, d, False, signs=bits)
+    assert err == 0
+    ek, ev = ora.encode(x, bits), ora.encode(x[::-1], bits)
+    assert np.array_equal(kb, ora.pack_blocks(ek.codes, ek.scale_bits))
+    assert np.array_equal(vb, ora.pack_value_blocks(ev.codes, ev.scale_bits))
+    assert not np.array_equal(ek.codes, ora.encode(x).codes)  # the signs change the codes
 
 
 def test_encode_refusals_flag_and_zero_encode(akv, wlmod, cuda):
@@ -227,6 +241,7 @@ def test_exact_gqa_full_size(akv, wlmod, cuda, variant):
 
 def _oracle_hybrid(wl, w, b, heads=None):
     """Oracle for sequence b of a HybridResident: encode the old part, dequantise, attend."""
+    bits = getattr(w, "rotation_signs", 0)
     Tc = w.T - w.W
     kk = w.k_bits[b]
     vv = w.v_bits[b]
@@ -235,10 +250,10 @@ def _oracle_hybrid(wl, w, b, heads=None):
     vh = np.zeros((H, Tc, wl.d))
     codes = []
     for h in range(H):
-        ek = ora.encode(kk[h, :Tc])
-        ev = ora.encode(vv[h, :Tc])
-        kh[h] = ora.dequantize(ek.codes, ek.scale_bits)
-        vh[h] = ora.dequantize(ev.codes, ev.scale_bits)
+        ek = ora.encode(kk[h, :Tc], bits)
+        ev = ora.encode(vv[h, :Tc], bits)
+        kh[h] = ora.dequantize(ek.codes, ek.scale_bits, bits)
+        vh[h] = ora.dequantize(ev.codes, ev.scale_bits, bits)
         codes.append((ora.pack_blocks(ek.codes, ek.scale_bits), ora.pack_value_blocks(ev.codes, ev.scale_bits)))
     tiers = [(kh, vh), (f64(kk[:, Tc:]), f64(vv[:, Tc:]))]
     return ora.decode_sequence(f64(w.q_bits[b]), tiers, wl.scale, wl.split_tokens), codes
@@ -260,6 +275,25 @@ def test_hybrid_small(akv, wlmod, cuda, variant, T, W, d, G):
             assert np.array_equal(kc[b, h], codes[h][0]) and np.array_equal(vc[b, h], codes[h][1])
         check_partials(w.step, 0, b, partials[0])
         check_partials(w.step, 1, b, partials[1])
+        check_merged(w.step, b, direct)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("T,W,d,G", [(2600, 600, 128, 4), (1100, 300, 64, 8)])
+def test_hybrid_rotation_signs(akv, wlmod, cuda, variant, T, W, d, G):
+    """A randomised-sign rotation: codes, partials and merged output against the oracle."""
+    import torch
+    wl = synth.Workload("hybrid-signs", B=2, Hq=2 * G, Hkv=2, d=d, split_tokens=256, extra={"T": T, "window": W})
+    w = wlmod.HybridResident(wl, cuda, rotation_signs=synth.rotation_sign_bits(1, d))
+    w.step.step(w.q, variant_id(akv, variant))
+    torch.cuda.synchronize()
+    assert int(w.enc_err.item()) == 0
+    kc, vc = w.kc.cpu().numpy(), w.vc.cpu().numpy()
+    for b in range(w.B):
+        (partials, merged, direct), codes = _oracle_hybrid(wl, w, b)
+        for h in range(wl.Hkv):
+            assert np.array_equal(kc[b, h], codes[h][0]) and np.array_equal(vc[b, h], codes[h][1])
+        check_partials(w.step, 0, b, partials[0])
         check_merged(w.step, b, direct)
 
 
