@@ -140,6 +140,19 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                : "r"(a), "n"(OFF));
   return v;
 }
+template <int OFF = 0>
+__device__ __forceinline__ float lds_half(uint32_t a) {  // one binary16 from a ring stage, as float
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1+%2];\n" : "=h"(v) : "r"(a), "n"(OFF));
+  return __half2float(__ushort_as_half(v));
+}
+// 8 x 8 transpose of 16-bit elements across the warp: lane (r, c) holding row r, columns
+// 2c, 2c + 1 receives row r of the transpose (column r, rows 2c, 2c + 1 of the input).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t lds32_const(uint32_t a) {
   uint32_t v;
   asm("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(a));
@@ -822,18 +835,25 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   // the scales of tokens 2tq, 2tq + 1 (+ 8), value code bytes of dims [DPT g, DPT g + DPT)
   // of tokens 2tq, 2tq + 1 (+ 8)
   const uint32_t koff = C::K_OFF + g * C::ROWB + KB * tq;
-  const uint32_t ksoff = C::KS_OFF + 4 * tq;  // the value scales sit at + VS_OFF - KS_OFF
+  const uint32_t ksoff = C::KS_OFF + 2 * g;  // token g's key scale; the value scales sit at + VS_OFF - KS_OFF
   const uint32_t voff = C::V_OFF + tq * D + C::US * (g ^ (D == 128 ? 2 * tq : 4 * (tq >> 1)));
   static_assert((NST & (NST - 1)) == 0, "stage index by mask");
   int gs = 0;  // this warp's global step; its stage is gs % NST
 
-  uint32_t qa[D / 16][4];
-  float kfac = 0.f;
+  // Score columns: G <= 4 -- column c < 4 is head c's high part, column c + 4 its residual;
+  // G = 8 -- columns are the heads, the residuals in a second product.  Lane (g, tq) holds
+  // the scores of heads hA = 2tq, hB = 2tq + 1 (mod 4 when G <= 4) at tokens g and g + 8;
+  // when G <= 4 lanes tq >= 2 duplicate lanes tq - 2.
+  constexpr int NQ = G <= 4 ? 1 : 2;
+  const int hA = G <= 4 ? (2 * tq) & 3 : 2 * tq, hB = hA + 1;
+  uint32_t qb[NQ][D / 16][2];  // B fragments of the query columns
+  float kfA = 0.f, kfB = 0.f;  // score factors of heads hA, hB
   int q_pair = -1;
 
-  // Base-2 scores of the step held in stage sa: sc[j][e] is head g at token 8j + 2tq + e,
-  // S^T = (H q) K_hat^T with the B fragments looked up straight from the code bytes, the
-  // high (row g) and residual (row g + 8) parts added, times the key scale.
+  // Base-2 scores of the step held in stage sa: sc[t][e] is head (hA, hB)[e] at token g + 8t.
+  // S (16 tokens x 8 columns) = K_hat Q^T: the A fragments (tokens g and g + 8 over the
+  // lane's dimension range) are looked up straight from the key code bytes; high and
+  // residual columns are added, then the key scale applied.
   auto scores = [&](uint32_t sa, float (&sc)[2][2]) {
     uint32_t wk[2][KB / 4];
     const uint32_t ka = sa + koff;
@@ -846,25 +866,28 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       wk[0][0] = a.x; wk[0][1] = a.y;
       wk[1][0] = b.x; wk[1][1] = b.y;
     }
-    float st[2][4];
+    float st[NQ][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int q = 0; q < NQ; ++q)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st[j][e] = 0.f;
+      for (int e = 0; e < 4; ++e) st[q][e] = 0.f;
 #pragma unroll
-    for (int kc = 0; kc < D / 16; ++kc)
+    for (int kc = 0; kc < D / 16; ++kc) {
+      const uint32_t w0 = wk[0][kc >> 1], w1 = wk[1][kc >> 1];
+      const int bt = 2 * (kc & 1);
+      const uint32_t a[4] = {lookup(w0, bt), lookup(w1, bt), lookup(w0, bt + 1), lookup(w1, bt + 1)};
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t wd = wk[j][kc >> 1];
-        mma_f16(st[j], qa[kc], lookup(wd, 2 * (kc & 1)), lookup(wd, 2 * (kc & 1) + 1));
-      }
-    const uint32_t ksw[2] = {lds32<0>(sa + ksoff), lds32<16>(sa + ksoff)};
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float2 kh = unpack_f16(ksw[j]);
-      sc[j][0] = (st[j][0] + st[j][2]) * (kfac * kh.x);
-      sc[j][1] = (st[j][1] + st[j][3]) * (kfac * kh.y);
+      for (int q = 0; q < NQ; ++q) mma_f16(st[q], a, qb[q][kc][0], qb[q][kc][1]);
     }
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      v[e] = NQ == 1 ? st[0][e] + __shfl_xor_sync(kFull, st[0][e], 2) : st[0][e] + st[NQ - 1][e];
+    const float ks0 = lds_half<0>(sa + ksoff), ks8 = lds_half<16>(sa + ksoff);
+    sc[0][0] = v[0] * (kfA * ks0);
+    sc[0][1] = v[1] * (kfB * ks0);
+    sc[1][0] = v[2] * (kfA * ks8);
+    sc[1][1] = v[3] * (kfB * ks8);
   };
 
   for (int item = lo; item < hi; ++item) {
@@ -896,7 +919,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
 #pragma unroll
         for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], off));
       __syncwarp();  // earlier reads of the scratch are done
-      int my_e = 0;
+      int eA = 0, eB = 0;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         int e = 0;
@@ -910,21 +933,31 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
           sts32(scr(h * D + P * lane + j), hw);
           sts32(scr(h * D + P * lane + j + 1), pack_f16(x0 - hv.x, x1 - hv.y));
         }
-        if (g == h) my_e = e;
+        if (h == hA) eA = e;
+        if (h == hB) eB = e;
       }
       __syncwarp();
-      // lane (g, tq), step kc covers dims 2*KB*tq + 4kc + {0,1,2,3}: rows g = high parts,
-      // rows g + 8 = residuals
-      const int i0 = (g < G ? g : 0) * D + 2 * KB * tq;
+      // column g, step kc: dims 2*KB*tq + 4kc + {0, 1} (b0) and + {2, 3} (b1) of the lane's
+      // k range; the scratch holds (high, residual) word pairs per two dims
+      const int hg = G <= 4 ? (g & 3) : g;
+      const bool on = hg < G;
+      const int i0 = (on ? hg : 0) * D + 2 * KB * tq;
 #pragma unroll
       for (int kc = 0; kc < D / 16; ++kc) {
         const uint4 v = lds128<0>(scr(i0 + 4 * kc));
-        qa[kc][0] = g < G ? v.x : 0u;  // high, dims 4kc, 4kc+1
-        qa[kc][1] = g < G ? v.y : 0u;  // residual
-        qa[kc][2] = g < G ? v.z : 0u;  // high, dims 4kc+2, 4kc+3
-        qa[kc][3] = g < G ? v.w : 0u;  // residual
+        if constexpr (NQ == 1) {
+          const bool lo_part = g >= 4;
+          qb[0][kc][0] = on ? (lo_part ? v.y : v.x) : 0u;
+          qb[0][kc][1] = on ? (lo_part ? v.w : v.z) : 0u;
+        } else {
+          qb[0][kc][0] = v.x;
+          qb[0][kc][1] = v.z;
+          qb[NQ - 1][kc][0] = v.y;
+          qb[NQ - 1][kc][1] = v.w;
+        }
       }
-      kfac = p.scale_log2 / (float)D * ldexpf(1.f, my_e);
+      kfA = p.scale_log2 / (float)D * ldexpf(1.f, eA);
+      kfB = p.scale_log2 / (float)D * ldexpf(1.f, eB);
       __syncwarp();
     }
 
@@ -933,7 +966,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_A = -INFINITY, m_B = -INFINITY, l_A = 0.f, l_B = 0.f;  // heads hA, hB
     const int nsteps = (it.n + 15) >> 4;
     // Commit groups are counted in steps: before step S of this warp NST + S groups have been
     // committed, so waiting down to NST - 1 pending lands step S, and down to NST - 2 lands
@@ -952,42 +985,71 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       const int nv = min(16, it.n - 16 * s);
       if (nv < 16) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-            if (8 * j + 2 * tq + e >= nv) sc[j][e] = -INFINITY;
+        for (int t = 0; t < 2; ++t)
+          if (g + 8 * t >= nv) sc[t][0] = sc[t][1] = -INFINITY;
       }
       // the next step's scores, so their loads, lookups and MMAs overlap this step's
       // softmax and value product (after an item's last step the next stage holds the
       // following item's first step or nothing; those scores are not used)
       scores(nxt, sc_n);
-      float a_even, a_odd;
-      if (online_softmax<G>(sc, m_run, l_run, a_even, a_odd)) {
+      // ---- online softmax per head over the 16 tokens (2 per lane, 8 lane groups).  The
+      // reference m of each head sits kSlack above a maximum already seen, so the weights
+      // 2^(s - m) stay at most 1; only a score above m (in practice a split's first steps)
+      // costs the cross-lane maximum and the rescale.  LSE = m + log2 l holds for any m.
+      constexpr float kSlack = 8.f;
+      float mxA = fmaxf(sc[0][0], sc[1][0]), mxB = fmaxf(sc[0][1], sc[1][1]);
+      if (__any_sync(kFull, mxA > m_A || mxB > m_B)) {
 #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          acc[mt][0] *= a_even; acc[mt][1] *= a_odd;
-          acc[mt][2] *= a_even; acc[mt][3] *= a_odd;
+        for (int off = 4; off < 32; off <<= 1) {
+          mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, off));
+          mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, off));
         }
-      }
-      // ---- P' = P * s^V (0 for masked tokens): FP16 high part and residual
-      const uint32_t vsw[2] = {lds32<C::VS_OFF - C::KS_OFF>(st_s + ksoff),
-                               lds32<C::VS_OFF - C::KS_OFF + 16>(st_s + ksoff)};
-      float wts[2][2];
+        const float nA = fmaxf(m_A, mxA + kSlack), nB = fmaxf(m_B, mxB + kSlack);
+        const float aA = fast_exp2(m_A - nA), aB = fast_exp2(m_B - nB);  // 0 while m = -inf
+        l_A *= aA;
+        l_B *= aB;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float2 vh = unpack_f16(vsw[j]);
-        wts[j][0] = sc[j][0] * vh.x;
-        wts[j][1] = sc[j][1] * vh.y;
+        for (int mt = 0; mt < D / 16; ++mt) {  // accumulator columns 2tq, 2tq + 1 are heads hA, hB
+          acc[mt][0] *= aA; acc[mt][1] *= aB;
+          acc[mt][2] *= aA; acc[mt][3] *= aB;
+        }
+        m_A = nA;
+        m_B = nB;
       }
+      float w[2][2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        w[t][0] = fast_exp2(sc[t][0] - m_A);
+        w[t][1] = fast_exp2(sc[t][1] - m_B);
+      }
+      l_A += w[0][0] + w[1][0];
+      l_B += w[0][1] + w[1][1];
+      // ---- P' = P * s^V as the value product's B fragments.  Lane (g, tq) holds P' of tokens
+      // g, g + 8 at columns 2tq, 2tq + 1 (G <= 4: lanes tq < 2 the FP16 high parts, tq >= 2 the
+      // residuals); a transpose per 8 tokens gives column g at tokens 2tq, 2tq + 1 (+ 8).
+      const float vs0 = lds_half<C::VS_OFF - C::KS_OFF>(st_s + ksoff);
+      const float vs8 = lds_half<C::VS_OFF - C::KS_OFF + 16>(st_s + ksoff);
+      w[0][0] *= vs0; w[0][1] *= vs0;
+      w[1][0] *= vs8; w[1][1] *= vs8;
       if (nv < 16) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-            if (8 * j + 2 * tq + e >= nv) wts[j][e] = 0.f;
+        for (int t = 0; t < 2; ++t)
+          if (g + 8 * t >= nv) w[t][0] = w[t][1] = 0.f;
       }
       uint32_t pb[2], pl[2];
-      p_fragments<G, false>(wts, pb, pl);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint32_t hi = pack_f16(w[t][0], w[t][1]);
+        const float2 hv = unpack_f16(hi);
+        const uint32_t lo = pack_f16(w[t][0] - hv.x, w[t][1] - hv.y);
+        if constexpr (NQ == 1) {
+          pb[t] = transpose8x8(tq >= 2 ? lo : hi);
+          pl[t] = 0u;
+        } else {
+          pb[t] = transpose8x8(hi);
+          pl[t] = transpose8x8(lo);
+        }
+      }
       // ---- O_rot^T += V_hat^T P'^T: lane (g, tq) reads value dims [DPT g, DPT g + DPT) of
       // token pairs (2tq, 2tq+1) (pair row tq) and (2tq+8, 2tq+9) (pair row 4 + tq); byte k
       // of those words is dim DPT g + k of both tokens, so one lookup is one A-fragment entry
@@ -1019,15 +1081,19 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       ++gs;
     }
 
-    // ---- epilogue: O = H (acc / l) / D per head, LSE = ln 2 (m + log2 l)
-    l_run += __shfl_xor_sync(kFull, l_run, 1);
-    l_run += __shfl_xor_sync(kFull, l_run, 2);
-    if (tq == 0 && g < G)
-      p.lse_part[(size_t)it.slot * p.Hq + it.kvh * G + g] = kLn2 * (m_run + log2f(l_run));
-    const float inv_l = 1.f / ((float)D * l_run);
-    constexpr int HM = G <= 4 ? 3 : 7;
-    const float f_even = __shfl_sync(kFull, inv_l, ((2 * tq) & HM) * 4);
-    const float f_odd = __shfl_sync(kFull, inv_l, ((2 * tq + 1) & HM) * 4);
+    // ---- epilogue: l per head over the 8 lane groups, O = s . H (acc / l) / D per head,
+    // LSE = ln 2 (m + log2 l)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l_A += __shfl_xor_sync(kFull, l_A, off);
+      l_B += __shfl_xor_sync(kFull, l_B, off);
+    }
+    if (g == 0 && (G > 4 || tq < 2)) {
+      float* lse = p.lse_part + (size_t)it.slot * p.Hq + it.kvh * G;
+      if (hA < G) lse[hA] = kLn2 * (m_A + log2f(l_A));
+      if (hB < G) lse[hB] = kLn2 * (m_B + log2f(l_B));
+    }
+    const float f_even = 1.f / ((float)D * l_A), f_odd = 1.f / ((float)D * l_B);
     if constexpr (G <= 4) {  // fold the residual columns 4..7 into heads 0..3
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt)
