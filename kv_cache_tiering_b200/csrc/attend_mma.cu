@@ -246,36 +246,42 @@ __device__ __forceinline__ void cursor_next(const AttendParams& p, Cursor& c, in
 
 // ------------------------------------------------------------------------------------
 // online softmax of one step.  sc[j][e] (e < 2): base-2 scores of head g for tokens
-// 8j + 2tq + e, masked with -inf.  Leaves the weights in sc[j][e] and returns the rescale
-// factors of the accumulator columns 2tq, 2tq + 1 (column c holds head c for G = 8 and
-// head c % 4 for G <= 4).  Returns false when no rescale is needed (all factors 1, or the
-// chain's first step, whose accumulators are still zero).
+// 8j + 2tq + e, masked with -inf.  The running reference m_run of a head sits kSlack above
+// a maximum already seen, so the weights 2^(s - m_run) stay at most 1; only a score above
+// m_run (in practice a chain's first steps) costs the cross-lane maximum, and then the
+// function returns true with the rescale factors of the accumulator columns 2tq, 2tq + 1
+// (column c holds head c for G = 8 and head c % 4 for G <= 4).  LSE = m_run + log2 l_run
+// holds for any reference.  Leaves the weights in sc[j][e].
 // ------------------------------------------------------------------------------------
 template <int G, int N>
 __device__ __forceinline__ bool online_softmax(float (&sc)[2][N], float& m_run, float& l_run, float& a_even,
                                                float& a_odd) {
+  constexpr float kSlack = 8.f;
   const int lane = threadIdx.x & 31, tq = lane & 3;
   float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-  mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-  const float m_new = fmaxf(m_run, mx);
-  const bool grow = m_new > m_run && m_run != -INFINITY;  // a chain's first step has nothing to rescale
-  const float alpha = fast_exp2(m_run - m_new);  // 0 on a chain's first step (m_run = -inf)
+  bool rescale = false;
+  if (__any_sync(kFull, mx > m_run)) {
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float m_new = fmaxf(m_run, mx + kSlack);
+    const float alpha = fast_exp2(m_run - m_new);  // 0 while m_run = -inf
+    l_run *= alpha;
+    m_run = m_new;
+    constexpr int HM = G <= 4 ? 3 : 7;
+    a_even = __shfl_sync(kFull, alpha, ((2 * tq) & HM) * 4);
+    a_odd = __shfl_sync(kFull, alpha, ((2 * tq + 1) & HM) * 4);
+    rescale = true;
+  }
   float s = 0.f;
 #pragma unroll
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      sc[j][e] = fast_exp2(sc[j][e] - m_new);
+      sc[j][e] = fast_exp2(sc[j][e] - m_run);
       s += sc[j][e];
     }
-  l_run = l_run * alpha + s;
-  m_run = m_new;
-  if (!__any_sync(kFull, grow)) return false;
-  constexpr int HM = G <= 4 ? 3 : 7;
-  a_even = __shfl_sync(kFull, alpha, ((2 * tq) & HM) * 4);
-  a_odd = __shfl_sync(kFull, alpha, ((2 * tq + 1) & HM) * 4);
-  return true;
+  l_run += s;
+  return rescale;
 }
 
 // P^T B fragments from the weights w[j][e] (head g, tokens 8j + 2tq + e): high part and
