@@ -441,6 +441,71 @@ __device__ __forceinline__ void merge_tail(const AttendParams& p, const Item& it
   }
 }
 
+// The same merge by a whole CTA of NT threads, through shared memory `sm` (at least
+// 2 G + max(NT, G kTailChunk) floats; every thread of the CTA calls it).  Pass 1 finds each head's
+// maximum LSE over the sequence's slots; pass 2 takes the slots in chunks: their weights
+// exp(lse - M) go to shared memory, then every thread accumulates its outputs over the
+// chunk with independent loads.  Same formula and slot order as merge_tail.
+constexpr int kTailChunk = 64;
+template <int D, int G, int NT>
+__device__ void merge_tail_cta(const AttendParams& p, const Item& it, float* sm) {
+  static_assert(NT % G == 0, "thread layout of the tail");
+  constexpr int E = (G * D + NT - 1) / NT;  // outputs per thread (the last ones may be past G D)
+  const int t = threadIdx.x;
+  const int base = p.seq.seq_slot_base[it.bl], n = p.seq.seq_n_slots[it.bl];
+  const float* lse_p = p.lse_part + (size_t)base * p.Hq + it.kvh * G;
+  float* Mh = sm;             // [G]
+  float* Lh = sm + G;         // [G]
+  float* wsm = sm + 2 * G;    // [kTailChunk][G]
+  // pass 1: maxima (thread t takes head t % G, slots t / G, t / G + NT / G, ...)
+  float m = -INFINITY;
+  for (int s = t / G; s < n; s += NT / G) m = fmaxf(m, __ldcg(lse_p + (size_t)s * p.Hq + t % G));
+  wsm[t] = m;
+  __syncthreads();
+  if (t < G) {
+    float M = -INFINITY;
+    for (int k = t; k < NT; k += G) M = fmaxf(M, wsm[k]);
+    Mh[t] = M;
+  }
+  __syncthreads();
+  // pass 2: weights per chunk, then the weighted sums
+  float o[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o[e] = 0.f;
+  float L = 0.f;
+  for (int c0 = 0; c0 < n; c0 += kTailChunk) {
+    const int nc = min(kTailChunk, n - c0);
+    for (int k = t; k < nc * G; k += NT) {
+      const int h = k % G;
+      wsm[k] = Mh[h] == -INFINITY ? 0.f : expf(__ldcg(lse_p + (size_t)(c0 + k / G) * p.Hq + h) - Mh[h]);
+    }
+    __syncthreads();
+    if (t < G)
+      for (int s = 0; s < nc; ++s) L += wsm[s * G + t];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = t + e * NT, h = i / D, dim = i % D;
+      if (i >= G * D) break;
+      const float* op = p.o_part + ((size_t)(base + c0) * p.Hq + it.kvh * G + h) * D + dim;
+      float a = o[e];
+#pragma unroll 8
+      for (int s = 0; s < nc; ++s) a = fmaf(wsm[s * G + h], __ldcg(op + (size_t)s * p.Hq * D), a);
+      o[e] = a;
+    }
+    __syncthreads();
+  }
+  if (t < G) Lh[t] = L;
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = t + e * NT, h = i / D, dim = i % D, hq = it.kvh * G + h;
+    if (i >= G * D) break;
+    const float M = Mh[h];
+    p.o[((size_t)it.b * p.Hq + hq) * D + dim] = M == -INFINITY ? 0.f : o[e] / Lh[h];
+    if (dim == 0) p.lse[(size_t)it.b * p.Hq + hq] = M == -INFINITY ? -INFINITY : M + logf(Lh[h]);
+  }
+}
+
 // Count a finished item; true for the caller that completed the (sequence, KV head).
 __device__ __forceinline__ bool finish_item(const AttendParams& p, const Item& it) {
   const int old = atomicAdd(p.counters + (size_t)it.b * p.Hkv + it.kvh, 1);
@@ -644,9 +709,9 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
       group_sync<NW>(gi);
       if (threadIdx.x == 0) *flag = finish_item(p, it) ? 1 : 0;
       group_sync<NW>(gi);
-      if (*flag) {
+      if (*flag) {  // CTA-uniform
         __threadfence();
-        merge_tail<D, G>(p, it, threadIdx.x, NW * 32);
+        merge_tail_cta<D, G, NW * 32>(p, it, area);
         if (threadIdx.x == 0) p.counters[(size_t)it.b * p.Hkv + it.kvh] = 0;
       }
     }
