@@ -61,6 +61,8 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+SAMPLE = 8  # timed steps between two steps whose launches are bracketed by events
+
 KERNEL_SOURCES = ("kv_cache_tiering_b200/csrc/attend_mma.cu", "kv_cache_tiering_b200/csrc/akv_internal.cuh")
 
 
@@ -385,11 +387,14 @@ def run_ours(args):
             one_step()
         torch.cuda.synchronize()
 
-    # events around every tier's launch, so the dominant kernel is timed on its own
+    # events around every tier's launch on every SAMPLE-th step, so the dominant kernel is
+    # timed on its own; the other steps run without events between their launches (an event
+    # between two kernels would stop the next one from overlapping the previous one's tail)
     live = [i for i, t in enumerate(step.tiers) if int(sum(t.lens)) > 0]
     per_tier = not fuse and len(live) > 1
     n_b = len(live) + 1 if per_tier else 2
-    bounds = [[torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] for _ in range(n_b)]
+    sampled = list(range(0, args.steps, SAMPLE))
+    bounds = [[torch.cuda.Event(enable_timing=True) for _ in sampled] for _ in range(n_b)]
     a0, a1 = bounds[0], bounds[-1]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
@@ -400,16 +405,19 @@ def run_ours(args):
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(1)
-        a0[i].record(stream)
+        k = i // SAMPLE if i % SAMPLE == 0 else -1
+        if k >= 0:
+            a0[k].record(stream)
         if fuse:
             step.decode(w.q, variant, stream)
-        elif per_tier:
+        elif per_tier and k >= 0:
             for j, ti in enumerate(live):
                 step.attend_tier(ti, w.q, variant, stream)
-                bounds[j + 1][i].record(stream)
+                bounds[j + 1][k].record(stream)
         else:
             step.attend(w.q, variant, stream)
-        a1[i].record(stream)
+        if k >= 0:
+            a1[k].record(stream)
         if not fuse:
             step.merge(stream)
     end.record(stream)
@@ -418,8 +426,8 @@ def run_ours(args):
     if dist:
         dist.barrier()
     ms = start.elapsed_time(end)
-    attend_ms = [a0[i].elapsed_time(a1[i]) for i in range(args.steps)]
-    tier_ms = ([statistics.fmean(bounds[j][i].elapsed_time(bounds[j + 1][i]) for i in range(args.steps))
+    attend_ms = [a0[k].elapsed_time(a1[k]) for k in range(len(sampled))]
+    tier_ms = ([statistics.fmean(bounds[j][k].elapsed_time(bounds[j + 1][k]) for k in range(len(sampled)))
                 for j in range(len(live))] if per_tier else None)
     if dist:
         ms = max_over_ranks(ms, dist, dev)

@@ -112,6 +112,13 @@ __device__ __forceinline__ int find_seq(const SeqTable& st, int item) {
   return lo;
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_overlapped may begin while
+// the previous kernel on its stream finishes: it lets its own successor be scheduled early,
+// does set-up that touches no global memory, then waits until the previous grid has
+// completed and its writes are visible -- before its first global read or write.
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void wait_prior_grids() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 __device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
   if (err) atomicOr(err, bits);
 }
@@ -129,7 +136,7 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
 // Physical page of logical page `lp` of global sequence b; out-of-pool ids are flagged
 // and replaced by page 0 so no access leaves the pool.
 __device__ __forceinline__ int64_t tier_page(const TierDev& t, int b, int lp, int32_t* err) {
-  int32_t p = __ldg(t.page_table + (int64_t)b * t.pt_stride + lp);
+  int32_t p = __ldcg(t.page_table + (int64_t)b * t.pt_stride + lp);
   if (p < 0 || (int64_t)p >= t.n_pages) {
     flag_error(err, AKV_EFLAG_BOUNDS);
     p = 0;
@@ -184,6 +191,24 @@ inline cudaError_t ensure_smem(int bytes) {
     }
   }
   return e;
+}
+
+// Launch `kernel` so that it may overlap the tail of the previous kernel on `s` (the kernel
+// must call wait_prior_grids before touching global memory).
+template <typename P>
+inline cudaError_t launch_overlapped(void (*kernel)(P), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                     const P& params) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, params);
 }
 
 // Streaming multiprocessors of the current device (queried once per device).

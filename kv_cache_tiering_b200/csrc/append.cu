@@ -15,7 +15,7 @@ __global__ void __launch_bounds__(32) append_kernel(const __grid_constant__ Appe
   const TierDev& t = p.tier;
   int64_t e;  // element offset of the destination row
   if (t.paged) {
-    const int32_t pg = __ldg(t.page_table + (int64_t)b * t.pt_stride + (pos >> 4));
+    const int32_t pg = __ldcg(t.page_table + (int64_t)b * t.pt_stride + (pos >> 4));
     if (pg < 0 || (int64_t)pg >= t.n_pages) {  // no write outside the pool
       if (lane == 0) flag_error(p.err, AKV_EFLAG_BOUNDS);
       return;

@@ -550,6 +550,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
   const uint32_t ring_s = smem_u32(smem + warp * NST * C::STAGE);
   const uint32_t bar_s = smem_u32(smem + C::BAR_OFF) + warp * NST * 8;
 
+  allow_next_grid();
   int lo, hi;
   cta_range(p.seq.item_base[p.seq.n_seq], lo, hi);
   if (lo >= hi) return;
@@ -559,6 +560,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
     fence_mbar_init();
   }
   __syncwarp();
+  wait_prior_grids();  // every global access comes after this
 
   // lane 0 fills stage st with step s of item it: one TMA box per 64-element half of K and V
   auto load_step = [&](const Item& it, int s, int st) {
@@ -796,7 +798,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const uint32_t base_s = smem_u32(smem);
   uint32_t lut_s, ring_s;
+  allow_next_grid();
   if (!codes_layout<C, NWARP>(base_s, warp, lut_s, ring_s)) {  // same answer in every thread
+    wait_prior_grids();
     if (threadIdx.x == 0) flag_error(p.err, AKV_EFLAG_INTERNAL);
     return;
   }
@@ -834,6 +838,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       }
     }
   };
+  // the lookup table is built from the launch parameters, before the wait for the previous
+  // grid; every global access comes after it
+  {
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_s - base_s));
+    for (int i = threadIdx.x; i < 256 * 32; i += NWARP * 32) {
+      const int byte = i >> 5, l = i & 31;
+      lut[byte * 64 + l] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
+    }
+  }
+  wait_prior_grids();
   uint32_t qw[G][P / 2];
   if (busy) load_q(item_at(p, lo), qw);
 
@@ -886,14 +900,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     }
   }
 
-  {
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_s - base_s));
-    for (int i = threadIdx.x; i < 256 * 32; i += NWARP * 32) {
-      const int byte = i >> 5, l = i & 31;
-      lut[byte * 64 + l] = (uint32_t)p.centroids[byte & 15] | ((uint32_t)p.centroids[byte >> 4] << 16);
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // the table is complete
   if (!busy) return;
 
   // table entry of byte `byte` of `word` for this lane: the table's own high address bytes,
@@ -1228,7 +1235,8 @@ cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   const int grid = n_items < sms ? n_items : sms;
-  k<<<grid, NW * 32, C::SMEM, s>>>(p);
+  e = launch_overlapped(k, dim3(grid), dim3(NW * 32), C::SMEM, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1242,7 +1250,8 @@ cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   const int grid = n_items < sms ? n_items : sms;
-  k<<<grid, NWARP * 32, C::SMEM, s>>>(p);
+  e = launch_overlapped(k, dim3(grid), dim3(NWARP * 32), C::SMEM, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   const int b = p.b0 + bl;
   const int base = p.slot_base[bl], n = p.n_slots[bl];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  allow_next_grid();
+  wait_prior_grids();  // the partials come from the attention launches before this one
 
   float M = -INFINITY, L = 0.f;
   float acc[P];
@@ -64,13 +66,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
     const int cn = min(kChunk, n - c0);
     float m = -INFINITY;
     for (int s = threadIdx.x; s < cn; s += kMergeThreads)
-      m = fmaxf(m, __ldg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h));
+      m = fmaxf(m, __ldcg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h));
     const float M_new = fmaxf(M, block_max(m, red));
     if (M_new == -INFINITY) continue;  // nothing finite so far
     const float r = expf(M - M_new);   // 0 while M is -inf
     float part = 0.f;
     for (int s = threadIdx.x; s < cn; s += kMergeThreads) {
-      const float w = expf(__ldg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h) - M_new);
+      const float w = expf(__ldcg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h) - M_new);
       wsh[s] = w;
       part += w;
     }
@@ -81,11 +83,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
       const float w = wsh[s];
       const float* row = p.o_part + ((size_t)(base + c0 + s) * p.Hq + h) * D + P * lane;
       if constexpr (P == 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(row));
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(row));
         acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
         acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
       } else {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(row));
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(row));
         acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
       }
     }
@@ -110,8 +112,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
 
 cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s) {
   dim3 grid(p.n_seq, p.Hq);
-  if (d == 128) merge_kernel<128><<<grid, kMergeThreads, 0, s>>>(p);
-  else merge_kernel<64><<<grid, kMergeThreads, 0, s>>>(p);
+  cudaError_t e = d == 128 ? launch_overlapped(merge_kernel<128>, grid, dim3(kMergeThreads), 0, s, p)
+                           : launch_overlapped(merge_kernel<64>, grid, dim3(kMergeThreads), 0, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
