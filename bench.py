@@ -439,26 +439,54 @@ def run_ours(args):
         torch.cuda.synchronize()
     err = int(step.err.item())
 
-    # ---- end to end through the public API: pinned host q in, O and LSE out, every step
+    # ---- end to end through the public API: every step copies its query in from pinned host
+    # memory and its O and LSE out to pinned host memory.  The copies run on streams of their
+    # own with two buffers each (events order every reuse), so a step's upload overlaps the
+    # previous step's compute and its download the next step's.
+    from kv_cache_tiering_b200 import workloads as wlmod
     q_host = torch.from_numpy(w.q_bits.view("int16")).pin_memory()
-    o_host = torch.empty(step.o.shape, dtype=torch.float32).pin_memory()
-    lse_host = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
-    q_dev = torch.empty_like(w.q)
-    for _ in range(3):
-        q_dev.copy_(q_host, non_blocking=True)
-        one_step()
+    pair = [step, wlmod.DecodeStep(step.B, step.Hq, step.Hkv, step.d, step.split_tokens, step.scale, step.tiers, dev)]
+    q_dev = [torch.empty_like(w.q) for _ in range(2)]
+    o_host = [torch.empty(step.o.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    lse_host = [torch.empty(step.lse.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # upload j landed
+    ev_used = [torch.cuda.Event() for _ in range(2)]  # step j's compute is done with its buffers
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # download j landed
+
+    def e2e_step(i):
+        j, st_j = i % 2, pair[i % 2]
+        up.wait_event(ev_used[j])
+        with torch.cuda.stream(up):
+            q_dev[j].copy_(q_host, non_blocking=True)
+            ev_in[j].record(up)
+        stream.wait_event(ev_in[j])
+        stream.wait_event(ev_out[j])
+        if flush is not None:
+            flush.fill_(1)
+        if fuse:
+            st_j.decode(q_dev[j], variant, stream)
+        else:
+            st_j.step(q_dev[j], variant, stream)
+        ev_used[j].record(stream)
+        down.wait_event(ev_used[j])
+        with torch.cuda.stream(down):
+            o_host[j].copy_(st_j.o, non_blocking=True)
+            lse_host[j].copy_(st_j.lse, non_blocking=True)
+            ev_out[j].record(down)
+
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     e0.record(stream)
-    for _ in range(args.steps):
-        q_dev.copy_(q_host, non_blocking=True)
-        if flush is not None:
-            flush.fill_(1)
-        run_step(q_dev)
-        o_host.copy_(step.o, non_blocking=True)
-        lse_host.copy_(step.lse, non_blocking=True)
+    up.wait_event(e0)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[(args.steps - 1) % 2])
+    stream.wait_event(ev_out[args.steps % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -505,7 +533,8 @@ def run_ours(args):
                              "attend_ms_avg": attend_avg_ms,
                              "tiers_ms_avg": dict(zip(kernel_names, tier_ms)) if per_tier else None},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(q_host.numel() * 2),
-                        "d2h_bytes_per_step": int(o_host.numel() * 4 + lse_host.numel() * 4)},
+                        "d2h_bytes_per_step": int(o_host[0].numel() * 4 + lse_host[0].numel() * 4),
+                        "pipelining": "copies on their own streams, two buffers each"},
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clocks, "device_error_word": err}
         if world == 1 and not args.no_cpu_baseline:
