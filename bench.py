@@ -282,10 +282,12 @@ def blas_threads():
 
 
 def time_oracle(name, wl, budget_s: float = 15.0, max_units=None):
+    """The oracle on a bounded sample: units of the workload (cycling through them) until
+    budget_s seconds or max_units units (default: 8 passes over the workload's units)."""
     fn, n_units, desc = oracle_sequence_fn(name, wl)
     tokens, units = 0.0, 0
     t0 = time.perf_counter()
-    while units < (max_units or n_units):
+    while units < (max_units or 8 * n_units):
         tokens += fn(units)
         units += 1
         if time.perf_counter() - t0 > budget_s:

@@ -172,3 +172,17 @@ def test_append_tokens_refusals(akv):
     assert e.value.status == akv.AKV_ERR_INVALID
     akv.akv_append_tokens(t, [-1, -5], 2, 8, 128, 0x3000, 0x4000)  # nothing to write: no launch
     assert akv.lib.akv_append_tokens(ctypes.byref(t.c()), None, 1, 8, 128, None, None, None, None) == akv.AKV_ERR_INVALID
+
+
+def test_header_is_plain_c():
+    """include/akv.h is a C header: it compiles as C11 with strict warnings."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = '#include "akv.h"\nint main(void) { akv_tier t; (void)t; return akv_abi_version() > 0 ? 0 : 1; }\n'
+    r = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-x", "c", "-",
+                        "-I", os.path.join(root, "include")], input=src, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
