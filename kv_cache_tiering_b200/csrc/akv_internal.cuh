@@ -234,7 +234,12 @@ inline int sm_count() {
 cudaError_t launch_encode(const EncodeParams& p, int d, int n_items, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, int d, int n_seq, cudaStream_t s);
 cudaError_t launch_attend_simt(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
-cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s);
+// Tensor-core split attention of one tier: a persistent grid of at most max_ctas CTAs (0: one
+// per SM); overlap = launched with programmatic stream serialization.
+cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s,
+                              int max_ctas = 0, bool overlap = true);
+// Warps per CTA of the compact-tier kernel for group size G (each runs one split at a time).
+int codes_warps_per_cta(int G);
 // Fill p.tmk / p.tmv for a BF16 tier of B sequences (tokens [0, max_len)): 4-D maps
 // (d, tokens, heads, sequences or pages), 64-element x 16-token boxes, 128-byte swizzle.
 cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int Hkv, int d, int64_t max_len);

@@ -335,6 +335,103 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
 
 }  // extern "C"
 
+namespace {
+
+// One planned attention launch: its parameters, tier kind, (split, KV head) items and the
+// tokens of its longest split.
+struct PlannedLaunch {
+  akv::AttendParams p;
+  int kind;
+  int items;
+  int64_t split_len;
+};
+
+// Whether a compact launch and a BF16 launch should share the GPU, and with how many CTAs
+// (one per SM) for the compact one.  Estimated durations: a compact split runs on one warp and
+// costs about 1.35 us per 16-token step on an SM that holds a full CTA; a BF16 split runs on one
+// CTA as 8 chains and costs about 1.8 us per chain step while every SM streams; a launch that
+// follows another costs about 4 us of ramp and tail (B200 measurements of the two kernels).
+// The share minimises the larger of the two durations (ties go to the smaller share, so the
+// BF16 tier keeps the slack); it is used only when that beats the two launches in a row, which
+// is when one of them would leave SMs or warps idle.  Returns 0 for "in a row".
+int compact_sm_share(int sms, int64_t items_c, int warps_c, int64_t steps_c, int64_t items_x, int64_t chain_steps_x) {
+  constexpr double kCodesStep = 1.35, kBf16ChainStep = 1.8, kLaunch = 4.0;
+  auto t_codes = [&](int ctas) { return (double)ceil_div(items_c, (int64_t)warps_c * ctas) * steps_c * kCodesStep; };
+  auto t_bf16 = [&](int ctas) { return (double)ceil_div(items_x, ctas) * chain_steps_x * kBf16ChainStep; };
+  int best = 0;
+  double best_t = t_codes(sms) + t_bf16(sms) + kLaunch;
+  for (int share = 1; share < sms; ++share) {
+    const double t = std::max(t_codes(share), t_bf16(sms - share));
+    if (t < best_t) {
+      best_t = t;
+      best = share;
+    }
+  }
+  return best;
+}
+
+// A second stream per device with a fork and a join event.  Created on first use and kept for
+// the life of the process; every enqueue sequence that uses it holds side_mutex().
+struct SideLane {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+std::mutex& side_mutex() {
+  static std::mutex m;
+  return m;
+}
+
+cudaError_t side_lane(SideLane*& out) {
+  static SideLane lanes[akv::kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= akv::kMaxDevices) return cudaErrorInvalidDevice;
+  SideLane& l = lanes[dev];
+  if (!l.stream) {
+    SideLane n;
+    if ((e = cudaStreamCreateWithFlags(&n.stream, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) == cudaSuccess &&
+        (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) == cudaSuccess) {
+      l = n;
+    } else {
+      if (n.fork) cudaEventDestroy(n.fork);
+      cudaStreamDestroy(n.stream);
+      return e;
+    }
+  }
+  out = &l;
+  return cudaSuccess;
+}
+
+// The compact launch c on the caller's stream with `share` CTAs, and the BF16 launch x on the
+// device's side stream with `rest` CTAs, so the two persistent grids hold disjoint SMs at the
+// same time.  The side stream starts after the work enqueued on `st` so far, and `st` resumes
+// after both launches; each split's arithmetic is independent of the grid, so the partials
+// are the same bits as from two launches in a row.
+akv_status side_by_side(const PlannedLaunch& c, const PlannedLaunch& x, int share, int rest, int d, int G,
+                        cudaStream_t st) {
+  std::lock_guard<std::mutex> lock(side_mutex());
+  SideLane* lane = nullptr;
+  cudaError_t e = side_lane(lane);
+  if (e != cudaSuccess) return cuda_fail(e, "side stream");
+  if ((e = cudaEventRecord(lane->fork, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(lane->stream, lane->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  const cudaError_t ex = akv::launch_attend_mma(x.p, d, G, x.kind, x.items, lane->stream, rest, false);
+  // the join is recorded and waited for even after a failed launch, so `st` never runs ahead of
+  // anything the side stream was given
+  if ((e = cudaEventRecord(lane->join, lane->stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  const cudaError_t ec =
+      ex == cudaSuccess ? akv::launch_attend_mma(c.p, d, G, c.kind, c.items, st, share, true) : cudaSuccess;
+  if ((e = cudaStreamWaitEvent(st, lane->join, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  if (ex != cudaSuccess) return cuda_fail(ex, "attend launch");
+  if (ec != cudaSuccess) return cuda_fail(ec, "attend launch");
+  return ok();
+}
+
+}  // namespace
+
 namespace akv {
 
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
@@ -378,30 +475,43 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
   p.counters = fused ? fused->counters : nullptr;
   p.o = fused ? fused->o : nullptr;
   p.lse = fused ? fused->lse : nullptr;
+  // every launch is planned (and every refusal made) before the first one is enqueued
+  const bool simt = variant == AKV_VARIANT_SIMT;
+  std::vector<PlannedLaunch> plan;
   for (int i = 0; i < n_tiers; ++i) {
     p.tier = tier_dev(&tiers[i]);
     for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
       const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
       // the CUDA-core kernels take a (split, KV head) grid; the tensor-core kernels a flat
       // list of (split, KV head) items
-      const bool simt = variant == AKV_VARIANT_SIMT;
       const int64_t items =
           fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv,
                          fused ? fused->seq_slot_base : nullptr, fused ? fused->seq_n_slots : nullptr);
       if (items == 0) continue;
       if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
+      int64_t max_len = 0;
+      for (int b = b0; b < b0 + n; ++b) max_len = std::max<int64_t>(max_len, tiers[i].lens[b]);
       if (!simt && tiers[i].kind == AKV_TIER_BF16) {
-        int64_t max_len = 0;
-        for (int b = b0; b < b0 + n; ++b) max_len = std::max<int64_t>(max_len, tiers[i].lens[b]);
         // global coordinates of the launch's sequences run up to b0 + n
         if (akv::make_bf16_tensor_maps(p, &tiers[i], b0 + n, Hkv, d, max_len) != cudaSuccess)
           return fail(AKV_ERR_UNSUPPORTED, "tier %d: cannot describe its layout to the tensor memory accelerator", i);
       }
-      // AUTO takes the tensor-core path, which measures faster on both tiers
-      cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
-                           : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
-      if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+      plan.push_back(PlannedLaunch{p, tiers[i].kind, (int)items, std::min<int64_t>(max_len, split_tokens)});
     }
+  }
+  const int sms = akv::sm_count();
+  if (!simt && plan.size() == 2 && plan[0].kind != plan[1].kind && sms >= 2) {
+    const PlannedLaunch& c = plan[0].kind == AKV_TIER_CODES4 ? plan[0] : plan[1];
+    const PlannedLaunch& x = plan[0].kind == AKV_TIER_CODES4 ? plan[1] : plan[0];
+    const int share = compact_sm_share(sms, c.items, akv::codes_warps_per_cta(G), ceil_div(c.split_len, 16), x.items,
+                                       ceil_div(ceil_div(x.split_len, 16), 8));
+    if (share > 0) return side_by_side(c, x, share, sms - share, d, G, st);
+  }
+  for (const PlannedLaunch& l : plan) {
+    // AUTO takes the tensor-core path, which measures faster on both tiers
+    cudaError_t e = simt ? akv::launch_attend_simt(l.p, d, G, l.kind, l.items, st)
+                         : akv::launch_attend_mma(l.p, d, G, l.kind, l.items, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attend launch");
   }
   return ok();
 }

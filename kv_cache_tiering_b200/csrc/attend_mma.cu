@@ -1226,58 +1226,64 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
 }
 
 template <int D, int G>
-cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s) {
+cudaError_t launch_bf16(const AttendParams& p, int n_items, cudaStream_t s, int max_ctas, bool overlap) {
   constexpr int NW = 8;
   constexpr int NST = G <= 4 ? 3 : 2;
   using C = Bf16Cfg<D, G, NW, NST>;
   auto k = attend_bf16_mma<D, G, NW, NST>;
   cudaError_t e = ensure_smem<attend_bf16_mma<D, G, NW, NST>>((int)C::SMEM);
   if (e != cudaSuccess) return e;
-  const int sms = sm_count();
-  const int grid = n_items < sms ? n_items : sms;
-  e = launch_overlapped(k, dim3(grid), dim3(NW * 32), C::SMEM, s, p);
+  const int ctas = max_ctas > 0 ? max_ctas : sm_count();
+  const int grid = n_items < ctas ? n_items : ctas;
+  e = overlap ? launch_overlapped(k, dim3(grid), dim3(NW * 32), C::SMEM, s, p)
+              : (k<<<grid, NW * 32, C::SMEM, s>>>(p), cudaSuccess);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int D, int G>
-cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s) {
+cudaError_t launch_codes(const AttendParams& p, int n_items, cudaStream_t s, int max_ctas, bool overlap) {
   constexpr int NWARP = G <= 4 ? 16 : 8;
   constexpr int NST = 4;
   using C = CodesCfg<D, G, NWARP, NST>;
   auto k = attend_codes_mma<D, G, NWARP, NST>;
   cudaError_t e = ensure_smem<attend_codes_mma<D, G, NWARP, NST>>((int)C::SMEM);
   if (e != cudaSuccess) return e;
-  const int sms = sm_count();
-  const int grid = n_items < sms ? n_items : sms;
-  e = launch_overlapped(k, dim3(grid), dim3(NWARP * 32), C::SMEM, s, p);
+  const int ctas = max_ctas > 0 ? max_ctas : sm_count();
+  const int grid = n_items < ctas ? n_items : ctas;
+  e = overlap ? launch_overlapped(k, dim3(grid), dim3(NWARP * 32), C::SMEM, s, p)
+              : (k<<<grid, NWARP * 32, C::SMEM, s>>>(p), cudaSuccess);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_d(const AttendParams& p, int G, int kind, int n_items, cudaStream_t s) {
+cudaError_t launch_d(const AttendParams& p, int G, int kind, int n_items, cudaStream_t s, int max_ctas, bool overlap) {
   if (kind == AKV_TIER_BF16) {
     switch (G) {
-      case 1: return launch_bf16<D, 1>(p, n_items, s);
-      case 2: return launch_bf16<D, 2>(p, n_items, s);
-      case 4: return launch_bf16<D, 4>(p, n_items, s);
-      default: return launch_bf16<D, 8>(p, n_items, s);
+      case 1: return launch_bf16<D, 1>(p, n_items, s, max_ctas, overlap);
+      case 2: return launch_bf16<D, 2>(p, n_items, s, max_ctas, overlap);
+      case 4: return launch_bf16<D, 4>(p, n_items, s, max_ctas, overlap);
+      default: return launch_bf16<D, 8>(p, n_items, s, max_ctas, overlap);
     }
   }
   switch (G) {
-    case 1: return launch_codes<D, 1>(p, n_items, s);
-    case 2: return launch_codes<D, 2>(p, n_items, s);
-    case 4: return launch_codes<D, 4>(p, n_items, s);
-    default: return launch_codes<D, 8>(p, n_items, s);
+    case 1: return launch_codes<D, 1>(p, n_items, s, max_ctas, overlap);
+    case 2: return launch_codes<D, 2>(p, n_items, s, max_ctas, overlap);
+    case 4: return launch_codes<D, 4>(p, n_items, s, max_ctas, overlap);
+    default: return launch_codes<D, 8>(p, n_items, s, max_ctas, overlap);
   }
 }
 
 }  // namespace
 
 // n_items counts (split, KV head) items: seq.item_base must count splits * Hkv.
-cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s) {
-  return d == 128 ? launch_d<128>(p, G, kind, n_items, s) : launch_d<64>(p, G, kind, n_items, s);
+cudaError_t launch_attend_mma(const AttendParams& p, int d, int G, int kind, int n_items, cudaStream_t s, int max_ctas,
+                              bool overlap) {
+  return d == 128 ? launch_d<128>(p, G, kind, n_items, s, max_ctas, overlap)
+                  : launch_d<64>(p, G, kind, n_items, s, max_ctas, overlap);
 }
+
+int codes_warps_per_cta(int G) { return G <= 4 ? 16 : 8; }
 
 }  // namespace akv

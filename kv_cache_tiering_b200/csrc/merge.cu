@@ -8,7 +8,9 @@
 //   3. warp w accumulates slots w, w + 8, ... of the chunk, lane l owning coordinates
 //      [P*l, P*l + P) (coalesced rows), and the eight warp sums are added in warp order.
 // Partial sums from an earlier chunk are rescaled by exp(M_old - M_new).  Every sum is taken
-// in a fixed order, so the result is deterministic.
+// in a fixed order, so the result is deterministic.  The kernel is bound by memory latency
+// (a few KB per CTA), so each thread's LSE values and each warp's first kRows partial rows of
+// a chunk are requested together, before the first reduction, and later rows kRows at a time.
 #include "akv_internal.cuh"
 
 namespace akv {
@@ -46,7 +48,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_constant__ MergeParams p) {
-  constexpr int P = D / 32;  // coordinates per lane
+  constexpr int P = D / 32;                          // coordinates per lane
+  constexpr int kPer = kChunk / kMergeThreads;       // LSE values per thread in a chunk
+  constexpr int kRows = 8;                           // partial rows in flight per warp
   __shared__ float wsh[kChunk];
   __shared__ float red[kMergeWarps];
   __shared__ float acc_sh[kMergeWarps][D];
@@ -61,34 +65,65 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
   float acc[P];
 #pragma unroll
   for (int j = 0; j < P; ++j) acc[j] = 0.f;
+  // rows of slots c0 + r0 + warp + kMergeWarps i (i < kRows) that lie below cn; zeros past it
+  float rows[kRows][P];
+  auto load_rows = [&](int c0, int r0, int cn) {
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const int s = r0 + warp + kMergeWarps * i;
+#pragma unroll
+      for (int j = 0; j < P; ++j) rows[i][j] = 0.f;
+      if (s < cn) {
+        const float* row = p.o_part + ((size_t)(base + c0 + s) * p.Hq + h) * D + P * lane;
+        if constexpr (P == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(row));
+          rows[i][0] = v.x; rows[i][1] = v.y; rows[i][2] = v.z; rows[i][3] = v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(row));
+          rows[i][0] = v.x; rows[i][1] = v.y;
+        }
+      }
+    }
+  };
 
   for (int c0 = 0; c0 < n; c0 += kChunk) {
     const int cn = min(kChunk, n - c0);
+    float ls[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int s = (int)threadIdx.x + kMergeThreads * k;
+      ls[k] = s < cn ? __ldcg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h) : -INFINITY;
+    }
+    load_rows(c0, 0, cn);
     float m = -INFINITY;
-    for (int s = threadIdx.x; s < cn; s += kMergeThreads)
-      m = fmaxf(m, __ldcg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h));
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) m = fmaxf(m, ls[k]);
     const float M_new = fmaxf(M, block_max(m, red));
     if (M_new == -INFINITY) continue;  // nothing finite so far
     const float r = expf(M - M_new);   // 0 while M is -inf
     float part = 0.f;
-    for (int s = threadIdx.x; s < cn; s += kMergeThreads) {
-      const float w = expf(__ldcg(p.lse_part + (size_t)(base + c0 + s) * p.Hq + h) - M_new);
-      wsh[s] = w;
-      part += w;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int s = (int)threadIdx.x + kMergeThreads * k;
+      if (s < cn) {
+        const float w = expf(ls[k] - M_new);
+        wsh[s] = w;
+        part += w;
+      }
     }
     L = L * r + block_sum(part, red);  // block_sum's barriers also publish wsh
 #pragma unroll
     for (int j = 0; j < P; ++j) acc[j] *= r;
-    for (int s = warp; s < cn; s += kMergeWarps) {
-      const float w = wsh[s];
-      const float* row = p.o_part + ((size_t)(base + c0 + s) * p.Hq + h) * D + P * lane;
-      if constexpr (P == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(row));
-        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
-        acc[2] = fmaf(w, v.z, acc[2]); acc[3] = fmaf(w, v.w, acc[3]);
-      } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(row));
-        acc[0] = fmaf(w, v.x, acc[0]); acc[1] = fmaf(w, v.y, acc[1]);
+    for (int r0 = 0; r0 < cn; r0 += kMergeWarps * kRows) {
+      if (r0 > 0) load_rows(c0, r0, cn);
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int s = r0 + warp + kMergeWarps * i;
+        if (s < cn) {
+          const float w = wsh[s];
+#pragma unroll
+          for (int j = 0; j < P; ++j) acc[j] = fmaf(w, rows[i][j], acc[j]);
+        }
       }
     }
     M = M_new;

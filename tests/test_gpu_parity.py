@@ -468,3 +468,36 @@ def test_fused_decode_refuses_small_workspace(akv, wlmod, cuda):
         akv.akv_decode(w.q, w.B, wl.Hq, wl.Hkv, wl.d, wl.scale, w.step.tiers, wl.split_tokens, w.step.workspace,
                        w.step.ws_bytes - 256, w.step.o, w.step.lse)
     assert e.value.status == akv.AKV_ERR_BUDGET
+
+
+@pytest.mark.parametrize("which", ["hybrid", "ragged"])
+def test_side_by_side_tiers_match_serial(akv, wlmod, cuda, which):
+    """One call over both tiers runs the compact and BF16 launches side by side on disjoint
+    SMs; its partials and merged outputs are the same bits as the two tiers launched one
+    after the other with full grids."""
+    import torch
+    if which == "hybrid":
+        w = wlmod.HybridResident(synth.WORKLOADS["hybrid"], cuda)
+    else:
+        wl = synth.Workload("ragged-side", B=12, Hq=32, Hkv=8, d=128, split_tokens=512,
+                            extra={"window": 1024, "nu": 3.0})
+        lens = np.array([700, 1024, 1025, 3000, 17, 5000, 9000, 2047, 1, 4096, 12000, 1500], np.int32)
+        w = wlmod.RaggedPaged(wl, cuda, lens=lens)
+    step = w.step
+    runs = []
+    for serial in (False, True, False):
+        step.o_part.fill_(float("nan"))
+        step.lse_part.fill_(float("nan"))
+        if serial:
+            for i in range(len(step.tiers)):
+                step.attend_tier(i, w.q)
+            step.merge()
+        else:
+            step.step(w.q)
+        torch.cuda.synchronize()
+        assert int(step.err.item()) == 0
+        runs.append([t.clone() for t in (step.o_part, step.lse_part, step.o, step.lse)])
+    for a, b in zip(runs[0], runs[1]):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    for a, b in zip(runs[0], runs[2]):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
