@@ -859,25 +859,31 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   static_assert(CH > 32 && CH <= 96, "at most three chunk rounds per block");
   int ld_item = lo, ld_left = 0;  // the loader's item and its steps not yet issued
   int ld_b = 0, ld_lp = 0;         // its sequence and the logical page of its next step
-  int64_t ld_blk = 0;              // contiguous: block of the next step; paged: the head's offset
+  // contiguous tiers: this lane's first chunk of the next key block, stepped by one token
+  // block per step; paged tiers: of the head's block in page 0.  A value block sits at a
+  // fixed distance from its key block.
+  const uint8_t* ld_k = nullptr;
+  const int64_t kv_delta = (int64_t)((uintptr_t)p.tier.v - (uintptr_t)p.tier.k);
+  const int64_t step_bytes = p.tier.s_tok * (int64_t)C::BLOCK;
+  const uint32_t lane16 = 16u * (uint32_t)lane;
   auto ld_begin = [&]() {
     const Item it = item_at(p, ld_item);
     ld_left = (it.n + 15) >> 4;
     ld_b = it.b;
     ld_lp = it.t0 >> 4;
-    ld_blk = (int64_t)it.kvh * p.tier.s_head;
-    if (!p.tier.paged) ld_blk += (int64_t)it.b * p.tier.s_seq + (int64_t)ld_lp * p.tier.s_tok;
+    int64_t blk = (int64_t)it.kvh * p.tier.s_head;
+    if (!p.tier.paged) blk += (int64_t)it.b * p.tier.s_seq + (int64_t)ld_lp * p.tier.s_tok;
+    ld_k = p.tier.k + blk * C::BLOCK + lane16;
   };
-  auto ld_issue = [&](int stage) {
-    int64_t blk = ld_blk;
+  auto ld_issue = [&](uint32_t stage_s) {  // fills the stage at shared address stage_s
+    const uint8_t* kb = ld_k;
     if (p.tier.paged) {
-      blk += tier_page(p.tier, ld_b, ld_lp, p.err) * p.tier.s_seq;
+      kb += tier_page(p.tier, ld_b, ld_lp, p.err) * p.tier.s_seq * (int64_t)C::BLOCK;
     } else {
-      ld_blk += p.tier.s_tok;
+      ld_k += step_bytes;
     }
-    const uint32_t dst = ring_s + stage * C::STAGE + 16 * lane;
-    const uint8_t* kb = p.tier.k + blk * C::BLOCK + 16 * lane;
-    const uint8_t* vb = p.tier.v + blk * C::BLOCK + 16 * lane;
+    const uint8_t* vb = kb + kv_delta;
+    const uint32_t dst = stage_s + lane16;
     cp_async16(dst + C::K_OFF, kb);
     cp_async16(dst + C::V_OFF, vb);
     if (CH >= 64 || 32 + lane < CH) {
@@ -895,7 +901,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     ld_begin();
 #pragma unroll
     for (int j = 0; j < NST; ++j) {
-      if (ld_item < hi) ld_issue(j);
+      if (ld_item < hi) ld_issue(ring_s + j * C::STAGE);
       cp_async_commit();
     }
   }
@@ -930,8 +936,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
 
   // Base-2 scores of the step held in stage sa: sc[t][e] is head (hA, hB)[e] at token g + 8t.
   // S (16 tokens x 8 columns) = K_hat Q^T: the A fragments (tokens g and g + 8 over the
-  // lane's dimension range) are looked up straight from the key code bytes; high and
-  // residual columns are added, then the key scale applied.
+  // lane's dimension range) are looked up straight from the key code bytes and accumulated
+  // as two independent chains (even and odd 16-dimension slices, so the products overlap);
+  // the chains, then the high and residual columns are added, then the key scale applied.
   auto scores = [&](uint32_t sa, float (&sc)[2][2]) {
     uint32_t wk[2][KB / 4];
     const uint32_t ka = sa + koff;
@@ -944,19 +951,23 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       wk[0][0] = a.x; wk[0][1] = a.y;
       wk[1][0] = b.x; wk[1][1] = b.y;
     }
-    float st[NQ][4];
+    float st[NQ][4], st_odd[NQ][4];
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) st[q][e] = 0.f;
+      for (int e = 0; e < 4; ++e) st[q][e] = st_odd[q][e] = 0.f;
 #pragma unroll
     for (int kc = 0; kc < D / 16; ++kc) {
       const uint32_t w0 = wk[0][kc >> 1], w1 = wk[1][kc >> 1];
       const int bt = 2 * (kc & 1);
       const uint32_t a[4] = {lookup(w0, bt), lookup(w1, bt), lookup(w0, bt + 1), lookup(w1, bt + 1)};
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) mma_f16(st[q], a, qb[q][kc][0], qb[q][kc][1]);
+      for (int q = 0; q < NQ; ++q) mma_f16((kc & 1) ? st_odd[q] : st[q], a, qb[q][kc][0], qb[q][kc][1]);
     }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[q][e] += st_odd[q][e];
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
@@ -1054,6 +1065,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     __syncwarp();
     scores(ring_s + (gs & (NST - 1)) * C::STAGE, sc_n);
 
+#pragma unroll 2  // fewer per-step moves and stage bookkeeping (measured)
     for (int s = 0; s < nsteps; ++s) {
       cp_async_wait<NST - 2>();  // this step and the next have landed
       __syncwarp();
@@ -1154,7 +1166,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         if constexpr (G > 4) mma_f16(acc[mt], a, pl[0], pl[1]);
       }
       __syncwarp();
-      if (ld_item < hi) ld_issue(gs & (NST - 1));  // refills the stage just read
+      if (ld_item < hi) ld_issue(st_s);  // refills the stage just read
       cp_async_commit();
       ++gs;
     }
