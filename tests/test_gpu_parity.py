@@ -501,3 +501,36 @@ def test_side_by_side_tiers_match_serial(akv, wlmod, cuda, which):
         assert torch.equal(a.view(torch.int32), b.view(torch.int32))
     for a, b in zip(runs[0], runs[2]):
         assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+@pytest.mark.parametrize("G,d", [(4, 128), (8, 64)])
+def test_hybrid_step_replays_from_cuda_graph(akv, wlmod, cuda, G, d):
+    """A decode step (the two tiers side by side, then the merge) captured into a CUDA graph
+    and replayed gives the same bits as the step run eagerly: the library's fork onto its
+    side stream and the join back are recorded as graph dependencies."""
+    import torch
+    wl = synth.Workload("hybrid-graph", B=3, Hq=8 * G, Hkv=8, d=d, split_tokens=512,
+                        extra={"T": 9000, "window": 2048})
+    w = wlmod.HybridResident(wl, cuda)
+    step = w.step
+    outs = (step.o, step.lse, step.o_part, step.lse_part)
+    s = torch.cuda.Stream(cuda)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step.step(w.q)  # eager; also creates the library's per-device state before capture
+    s.synchronize()
+    assert int(step.err.item()) == 0
+    ref = [t.clone() for t in outs]
+    for t in outs:
+        t.fill_(float("nan"))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step.step(w.q)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(step.err.item()) == 0
+        for a, b in zip(ref, outs):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    del g
