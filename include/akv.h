@@ -203,6 +203,14 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
  * variant and split layout the result does not depend on where the tokens are stored, so
  * a staged run equals the resident run bit for bit.  Page ids outside [0, n_pages) set
  * AKV_EFLAG_BOUNDS in *err_word (device, may be NULL) and read page 0 instead.
+ * Streams: asynchronous on `stream`; work enqueued on `stream` after the call sees every
+ * partial.  With one BF16 and one compact launch (tensor-core variants) the library may run
+ * the BF16 launch on an internal stream of the current device, forked from and joined back
+ * to `stream` with events, so the two grids share the SMs (same bits as launched in a row).
+ * That internal stream serves every such call on the device: a call whose `stream` is being
+ * captured into a graph must not run while another host thread enqueues such a call on the
+ * same device.  The first such call on a device creates the stream and its two events; make
+ * it before any capture.  Apart from an error message, no call allocates memory.
  * ------------------------------------------------------------------------------------ */
 enum { AKV_VARIANT_AUTO = 0, AKV_VARIANT_SIMT = 1, AKV_VARIANT_MMA = 2 };
 
@@ -260,7 +268,9 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
  *
  * The scratch is a fixed array of AKV_DECODE_STATIC_MAX_BYTES in this library's device
  * memory, held by every GPU that loads the library until the process exits; the call
- * itself allocates nothing, on the device or the host.  A step whose partials do not fit
+ * itself allocates no memory, on the device or the host (the first call that runs two tiers
+ * side by side creates the internal stream and events akv_decode_attend describes).  A step
+ * whose partials do not fit
  * (see akv_decode_workspace_size), or with more than AKV_DECODE_STATIC_MAX_SEQ sequences
  * or 8 tiers, returns AKV_ERR_BUDGET / AKV_ERR_UNSUPPORTED and launches nothing.  The
  * first call on each device looks up the array's device address while that device is

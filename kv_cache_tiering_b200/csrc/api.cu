@@ -480,40 +480,57 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
   p.counters = fused ? fused->counters : nullptr;
   p.o = fused ? fused->o : nullptr;
   p.lse = fused ? fused->lse : nullptr;
-  // every launch is planned (and every refusal made) before the first one is enqueued
+  // Every launch is checked (and every refusal made) before the first one is enqueued.  The
+  // first two launches are kept: that is all the side-by-side case needs, and a call with
+  // more launches rebuilds each one's parameters while enqueuing, so no call allocates.
   const bool simt = variant == AKV_VARIANT_SIMT;
-  std::vector<PlannedLaunch> plan;
-  for (int i = 0; i < n_tiers; ++i) {
-    p.tier = tier_dev(&tiers[i]);
-    for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
-      const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
-      // the CUDA-core kernels take a (split, KV head) grid; the tensor-core kernels a flat
-      // list of (split, KV head) items
-      const int64_t items =
-          fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv,
-                         fused ? fused->seq_slot_base : nullptr, fused ? fused->seq_n_slots : nullptr);
-      if (items == 0) continue;
-      if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
-      int64_t max_len = 0;
-      for (int b = b0; b < b0 + n; ++b) max_len = std::max<int64_t>(max_len, tiers[i].lens[b]);
-      if (!simt && tiers[i].kind == AKV_TIER_BF16) {
-        // global coordinates of the launch's sequences run up to b0 + n
-        if (akv::make_bf16_tensor_maps(p, &tiers[i], b0 + n, Hkv, d, max_len) != cudaSuccess)
-          return fail(AKV_ERR_UNSUPPORTED, "tier %d: cannot describe its layout to the tensor memory accelerator", i);
+  PlannedLaunch two[2];
+  int n_launch = 0;
+  // pass 0 checks and keeps, pass 1 (more than two launches) enqueues
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int i = 0; i < n_tiers; ++i) {
+      p.tier = tier_dev(&tiers[i]);
+      for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+        const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+        // the CUDA-core kernels take a (split, KV head) grid; the tensor-core kernels a flat
+        // list of (split, KV head) items
+        const int64_t items =
+            fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv,
+                           fused ? fused->seq_slot_base : nullptr, fused ? fused->seq_n_slots : nullptr);
+        if (items == 0) continue;
+        if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
+        int64_t max_len = 0;
+        for (int b = b0; b < b0 + n; ++b) max_len = std::max<int64_t>(max_len, tiers[i].lens[b]);
+        if (!simt && tiers[i].kind == AKV_TIER_BF16) {
+          // global coordinates of the launch's sequences run up to b0 + n
+          if (akv::make_bf16_tensor_maps(p, &tiers[i], b0 + n, Hkv, d, max_len) != cudaSuccess)
+            return fail(AKV_ERR_UNSUPPORTED, "tier %d: cannot describe its layout to the tensor memory accelerator",
+                        i);
+        }
+        if (pass == 0) {
+          if (n_launch < 2) two[n_launch] = PlannedLaunch{p, tiers[i].kind, (int)items, std::min<int64_t>(max_len, split_tokens)};
+          ++n_launch;
+        } else {
+          // AUTO takes the tensor-core path, which measures faster on both tiers
+          cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
+                               : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
+          if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+        }
       }
-      plan.push_back(PlannedLaunch{p, tiers[i].kind, (int)items, std::min<int64_t>(max_len, split_tokens)});
     }
+    if (pass == 0 && n_launch <= 2) break;
   }
+  if (n_launch > 2) return ok();
   const int sms = akv::sm_count();
-  if (!simt && plan.size() == 2 && plan[0].kind != plan[1].kind && sms >= 2) {
-    const PlannedLaunch& c = plan[0].kind == AKV_TIER_CODES4 ? plan[0] : plan[1];
-    const PlannedLaunch& x = plan[0].kind == AKV_TIER_CODES4 ? plan[1] : plan[0];
+  if (!simt && n_launch == 2 && two[0].kind != two[1].kind && sms >= 2) {
+    const PlannedLaunch& c = two[0].kind == AKV_TIER_CODES4 ? two[0] : two[1];
+    const PlannedLaunch& x = two[0].kind == AKV_TIER_CODES4 ? two[1] : two[0];
     const int share = compact_sm_share(sms, c.items, akv::codes_warps_per_cta(G), ceil_div(c.split_len, 16), x.items,
                                        ceil_div(ceil_div(x.split_len, 16), 8));
     if (share > 0) return side_by_side(c, x, share, sms - share, d, G, st);
   }
-  for (const PlannedLaunch& l : plan) {
-    // AUTO takes the tensor-core path, which measures faster on both tiers
+  for (int k = 0; k < n_launch; ++k) {
+    const PlannedLaunch& l = two[k];
     cudaError_t e = simt ? akv::launch_attend_simt(l.p, d, G, l.kind, l.items, st)
                          : akv::launch_attend_mma(l.p, d, G, l.kind, l.items, st);
     if (e != cudaSuccess) return cuda_fail(e, "attend launch");

@@ -288,6 +288,7 @@ class StagedDecode:
                 h = torch.empty((self.cap, 2, H, d), dtype=torch.int16).pin_memory()
                 h[: self.T, 0] = torch.from_numpy(k.view(np.int16))
                 h[: self.T, 1] = torch.from_numpy(v.view(np.int16))
+                h[self.T:].zero_()  # rows the appended tokens will take (a reused pinned block holds old data)
                 host_layers.append(h)
         self.host = host_layers
         self.copy_stream = torch.cuda.Stream(device)
