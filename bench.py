@@ -441,10 +441,11 @@ def run_ours(args):
         torch.cuda.synchronize()
     err = int(step.err.item())
 
-    # ---- end to end through the public API: every step copies its query in from pinned host
-    # memory and its O and LSE out to pinned host memory.  The copies run on streams of their
-    # own with two buffers each (events order every reuse), so a step's upload overlaps the
-    # previous step's compute and its download the next step's.
+    # ---- end to end through the public API: every step takes its query from pinned host memory
+    # and leaves O and LSE in pinned host memory.  Unfused, that is one akv_decode_host call
+    # per step on the compute stream (the GPU reads the query and writes the results over PCIe
+    # itself, alternating two output buffers).  Fused (akv_decode has no host form), the copies
+    # run on streams of their own with two buffers each, events ordering every reuse.
     from kv_cache_tiering_b200 import workloads as wlmod
     q_host = torch.from_numpy(w.q_bits.view("int16")).pin_memory()
     pair = [step, wlmod.DecodeStep(step.B, step.Hq, step.Hkv, step.d, step.split_tokens, step.scale, step.tiers, dev)]
@@ -456,7 +457,13 @@ def run_ours(args):
     ev_used = [torch.cuda.Event() for _ in range(2)]  # step j's compute is done with its buffers
     ev_out = [torch.cuda.Event() for _ in range(2)]   # download j landed
 
-    def e2e_step(i):
+    def e2e_host_step(i):
+        j = i % 2
+        if flush is not None:
+            flush.fill_(1)
+        step.decode_host(q_host, o_host[j], lse_host[j], 0, variant, stream)
+
+    def e2e_copy_step(i):
         j, st_j = i % 2, pair[i % 2]
         up.wait_event(ev_used[j])
         with torch.cuda.stream(up):
@@ -477,6 +484,7 @@ def run_ours(args):
             lse_host[j].copy_(st_j.lse, non_blocking=True)
             ev_out[j].record(down)
 
+    e2e_step = e2e_copy_step if fuse else e2e_host_step
     for i in range(4):
         e2e_step(i)
     torch.cuda.synchronize()
@@ -487,8 +495,9 @@ def run_ours(args):
     up.wait_event(e0)
     for i in range(args.steps):
         e2e_step(i)
-    stream.wait_event(ev_out[(args.steps - 1) % 2])
-    stream.wait_event(ev_out[args.steps % 2])
+    if fuse:
+        stream.wait_event(ev_out[(args.steps - 1) % 2])
+        stream.wait_event(ev_out[args.steps % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -536,7 +545,9 @@ def run_ours(args):
                              "tiers_ms_avg": dict(zip(kernel_names, tier_ms)) if per_tier else None},
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(q_host.numel() * 2),
                         "d2h_bytes_per_step": int(o_host[0].numel() * 4 + lse_host[0].numel() * 4),
-                        "pipelining": "copies on their own streams, two buffers each"},
+                        "transfers": ("copies on their own streams, two buffers each" if fuse else
+                                      "akv_decode_host: the GPU reads the pinned query and writes O and LSE "
+                                      "into pinned host memory, one stream")},
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clocks, "device_error_word": err}
         if world == 1 and not args.no_cpu_baseline:

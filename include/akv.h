@@ -259,6 +259,35 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
                       int variant, int32_t* err_word, akv_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * akv_decode_host -- one decode step with the query and the results in page-locked host
+ * memory: the end-to-end form of akv_decode_attend followed by akv_merge_lse.  No
+ * counterpart in the pages, which pass device tensors between their operators.
+ *
+ * q_host: page-locked host BF16 [B][Hq][d], 16-byte aligned.  o_host, lse_host:
+ * page-locked host float32 [B][Hq][d] and [B][Hq].  The call plans its own slots (the
+ * tiers' slot_base arrays are ignored) and enqueues on `stream`: the query copy into the
+ * workspace, the split attention of every tier, the merge, and the results into o_host and
+ * lse_host.  They are valid once that work has completed (synchronise the stream or an
+ * event recorded after the call); the host must not write q_host or read the outputs before.
+ * Transfers: where the driver reports that a host array lies wholly inside one page-locked
+ * allocation mapped for the device, the GPU reads the query over PCIe with a small kernel and
+ * the merge writes the outputs there directly, so the step's kernels overlap their launches;
+ * otherwise, or with flags AKV_HOST_COPY_ENGINE, the copy engine moves them.  Either way the
+ * results are the bits of akv_decode_attend + akv_merge_lse on the same inputs.
+ * workspace: caller-owned device scratch of at least akv_decode_host_workspace_size() bytes,
+ * 256-byte aligned; calls that share it must not overlap on the device.
+ * Refusals: a host array that is not page-locked -> AKV_ERR_NOT_PINNED; a small workspace
+ * -> AKV_ERR_BUDGET; the rest as akv_decode_attend.
+ * ------------------------------------------------------------------------------------ */
+#define AKV_HOST_COPY_ENGINE 0x1
+akv_status akv_decode_host_workspace_size(int B, int Hq, int Hkv, int d, const akv_tier* tiers, int n_tiers,
+                                          int split_tokens, size_t* bytes);
+akv_status akv_decode_host(const void* q_host, int B, int Hq, int Hkv, int d, float softmax_scale,
+                           const akv_tier* tiers, int n_tiers, int split_tokens, void* workspace,
+                           size_t workspace_bytes, float* o_host, float* lse_host, int flags, int variant,
+                           int32_t* err_word, akv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * akv_decode_static -- akv_decode without a workspace argument, for callers that cannot
  * allocate device memory when they decode (code inside a host function enqueued on a
  * stream, where CUDA forbids calls such as cudaMalloc; a plugin whose process memory pool

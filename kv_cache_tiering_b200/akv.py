@@ -38,6 +38,7 @@ AKV_TIER_CODES4 = 1
 AKV_VARIANT_AUTO = 0
 AKV_VARIANT_SIMT = 1
 AKV_VARIANT_MMA = 2
+AKV_HOST_COPY_ENGINE = 0x1
 PAGE_TOKENS = 16
 
 
@@ -105,6 +106,11 @@ _sig("akv_decode_workspace_size", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctyp
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t))
 _sig("akv_decode", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
      ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, _p, _p)
+_sig("akv_decode_host_workspace_size", ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t))
+_sig("akv_decode_host", ctypes.c_int, _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+     ctypes.POINTER(AkvTierC), ctypes.c_int, ctypes.c_int, _p, ctypes.c_size_t, _p, _p, ctypes.c_int, ctypes.c_int,
+     _p, _p)
 _sig("akv_append_tokens", ctypes.c_int, ctypes.POINTER(AkvTierC), _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p,
      _p, _p, _p)
 _sig("akv_checkpoint_write", ctypes.c_int, ctypes.c_char_p, ctypes.POINTER(ctypes.c_uint64), ctypes.c_int,
@@ -126,7 +132,7 @@ _sig("akv_stager_destroy", ctypes.c_int, _p)
 EXPORTED = [
     "akv_abi_version", "akv_last_error", "akv_status_string", "akv_error_word_status", "akv_centroids_f16",
     "akv_plan_slots", "akv_encode_history", "akv_decode_attend", "akv_merge_lse", "akv_decode_workspace_size",
-    "akv_decode", "akv_stager_create",
+    "akv_decode", "akv_decode_host_workspace_size", "akv_decode_host", "akv_stager_create",
     "akv_stage_chunk", "akv_stager_use", "akv_stager_release", "akv_stage_writeback", "akv_stager_destroy",
 ]
 
@@ -287,6 +293,23 @@ def akv_decode(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers
     ta = _tier_array(tiers)
     _check(lib.akv_decode(_ptr(q), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens, _ptr(workspace),
                           int(workspace_bytes), _ptr(o), _ptr(lse), variant, _ptr(err_word), _stream(stream)))
+
+
+def akv_decode_host_workspace_size(B: int, Hq: int, Hkv: int, d: int, tiers, split_tokens: int) -> int:
+    ta = _tier_array(tiers)
+    n = ctypes.c_size_t(0)
+    _check(lib.akv_decode_host_workspace_size(B, Hq, Hkv, d, ta.arr, ta.n, split_tokens, ctypes.byref(n)))
+    return n.value
+
+
+def akv_decode_host(q_host, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int,
+                    workspace, workspace_bytes: int, o_host, lse_host, flags: int = 0,
+                    variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
+    """One decode step with q_host, o_host and lse_host in page-locked host memory."""
+    ta = _tier_array(tiers)
+    _check(lib.akv_decode_host(_ptr(q_host), B, Hq, Hkv, d, float(softmax_scale), ta.arr, ta.n, split_tokens,
+                               _ptr(workspace), int(workspace_bytes), _ptr(o_host), _ptr(lse_host), flags, variant,
+                               _ptr(err_word), _stream(stream)))
 
 
 def akv_decode_static(q, B: int, Hq: int, Hkv: int, d: int, softmax_scale: float, tiers, split_tokens: int, o, lse,

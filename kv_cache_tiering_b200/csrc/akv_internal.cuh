@@ -244,6 +244,18 @@ int codes_warps_per_cta(int G);
 // (d, tokens, heads, sequences or pages), 64-element x 16-token boxes, 128-byte swizzle.
 cudaError_t make_bf16_tensor_maps(AttendParams& p, const akv_tier* t, int B, int Hkv, int d, int64_t max_len);
 cudaError_t launch_merge(const MergeParams& p, int d, cudaStream_t s);
+// Copy `bytes` (a multiple of 16) from host memory at device address src to dst, as a kernel
+// that reads at once and waits for the previous kernel on `s` only before writing.
+cudaError_t launch_copy_in(const void* src, void* dst, size_t bytes, cudaStream_t s);
+
+// Input copy a call enqueues after its checks and before its first attention launch: a
+// kernel reading mapped host memory (kernel = true) or a copy-engine transfer.
+struct CopyIn {
+  const void* src;
+  void* dst;
+  size_t bytes;
+  bool kernel;
+};
 
 // Fused decode: where the partials are merged.
 struct FusedArgs {
@@ -264,7 +276,8 @@ WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots)
 // Validated split attention of every tier (fused != null: merge folded in).
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused);
+                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused,
+                       const CopyIn* copy_in = nullptr);
 
 // Set the thread's last-error message; returns st.
 akv_status set_error(akv_status st, const char* msg);

@@ -141,6 +141,20 @@ WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots)
   return l;
 }
 
+PFN_cuPointerGetAttribute_v4000 pointer_attribute_fn() {
+  static PFN_cuPointerGetAttribute_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuPointerGetAttribute", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuPointerGetAttribute_v4000>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -435,13 +449,19 @@ akv_status side_by_side(const PlannedLaunch& c, const PlannedLaunch& x, int shar
   return ok();
 }
 
+akv_status enqueue_copy_in(const akv::CopyIn& c, cudaStream_t st) {
+  const cudaError_t e = c.kernel ? akv::launch_copy_in(c.src, c.dst, c.bytes, st)
+                                 : cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, st);
+  return e == cudaSuccess ? AKV_OK : cuda_fail(e, "query copy");
+}
+
 }  // namespace
 
 namespace akv {
 
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused) {
+                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused, const CopyIn* copy_in) {
   if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(AKV_ERR_INVALID, "Hq must be a positive multiple of Hkv");
   const int G = Hq / Hkv;
@@ -511,6 +531,11 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
           if (n_launch < 2) two[n_launch] = PlannedLaunch{p, tiers[i].kind, (int)items, std::min<int64_t>(max_len, split_tokens)};
           ++n_launch;
         } else {
+          if (copy_in) {
+            const akv_status cs = enqueue_copy_in(*copy_in, st);
+            if (cs != AKV_OK) return cs;
+            copy_in = nullptr;
+          }
           // AUTO takes the tensor-core path, which measures faster on both tiers
           cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
                                : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
@@ -521,6 +546,10 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
     if (pass == 0 && n_launch <= 2) break;
   }
   if (n_launch > 2) return ok();
+  if (copy_in) {  // nothing below refuses
+    const akv_status cs = enqueue_copy_in(*copy_in, st);
+    if (cs != AKV_OK) return cs;
+  }
   const int sms = akv::sm_count();
   if (!simt && n_launch == 2 && two[0].kind != two[1].kind && sms >= 2) {
     const PlannedLaunch& c = two[0].kind == AKV_TIER_CODES4 ? two[0] : two[1];
@@ -652,6 +681,122 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
   for (int b = 0; b < B && !need_merge; ++b) need_merge = sn[b] == 0;
   if (need_merge) return akv_merge_lse(o_part, lse_part, n_slots, sb.data(), sn.data(), B, Hq, d, o, lse, stream);
   return ok();
+}
+
+}  // extern "C"
+
+namespace {
+
+// Device view of a page-locked host array of `bytes` bytes at p: whether it is page-locked
+// host memory the device can address, and the device address of p; `whole` is set when all
+// of the array provably lies in that one allocation (the driver reports its range).
+struct HostArray {
+  bool pinned = false, whole = false;
+  void* dev = nullptr;
+};
+
+HostArray host_array(const void* p, size_t bytes) {
+  HostArray h;
+  cudaPointerAttributes a;
+  if (!p || cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return h;
+  }
+  h.pinned = a.type == cudaMemoryTypeHost;
+  if (!h.pinned || !a.devicePointer) return h;
+  h.dev = a.devicePointer;
+  auto get = akv::pointer_attribute_fn();
+  CUdeviceptr start = 0;
+  size_t size = 0;
+  if (get && get(&start, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, (CUdeviceptr)(uintptr_t)h.dev) == CUDA_SUCCESS &&
+      get(&size, CU_POINTER_ATTRIBUTE_RANGE_SIZE, (CUdeviceptr)(uintptr_t)h.dev) == CUDA_SUCCESS) {
+    const uintptr_t d0 = (uintptr_t)h.dev;
+    h.whole = start != 0 && size != 0 && d0 >= (uintptr_t)start && d0 - (uintptr_t)start <= size &&
+              bytes <= size - (d0 - (uintptr_t)start);
+  }
+  return h;
+}
+
+// Byte layout of an akv_decode_host workspace: the query copy, O and LSE (used when the
+// outputs go through the copy engine), the LSE partials, the O partials; 256-byte aligned.
+struct HostLayout {
+  size_t q, o, lse, lse_part, o_part, total;
+};
+
+HostLayout host_layout(int B, int Hq, int d, int64_t n_slots) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  HostLayout l;
+  l.q = 0;
+  l.o = up((size_t)B * Hq * d * 2);
+  l.lse = l.o + up((size_t)B * Hq * d * sizeof(float));
+  l.lse_part = l.lse + up((size_t)B * Hq * sizeof(float));
+  l.o_part = l.lse_part + up((size_t)n_slots * Hq * sizeof(float));
+  l.total = l.o_part + up((size_t)n_slots * Hq * d * sizeof(float));
+  return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+akv_status akv_decode_host_workspace_size(int B, int Hq, int Hkv, int d, const akv_tier* tiers, int n_tiers,
+                                          int split_tokens, size_t* bytes) {
+  if (!bytes) return fail(AKV_ERR_INVALID, "bytes is null");
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return fail(AKV_ERR_INVALID, "B >= 0, Hq, Hkv and d > 0 are required");
+  std::vector<std::vector<int32_t>> tb;
+  std::vector<int32_t> sb, sn;
+  int64_t n_slots = 0;
+  akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
+  if (s != AKV_OK) return s;
+  *bytes = host_layout(B, Hq, d, n_slots).total;
+  return ok();
+}
+
+akv_status akv_decode_host(const void* q_host, int B, int Hq, int Hkv, int d, float softmax_scale,
+                           const akv_tier* tiers, int n_tiers, int split_tokens, void* workspace,
+                           size_t workspace_bytes, float* o_host, float* lse_host, int flags, int variant,
+                           int32_t* err_word, akv_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "B >= 0, Hq and Hkv > 0 are required");
+  if (flags & ~AKV_HOST_COPY_ENGINE) return fail(AKV_ERR_INVALID, "unknown flags 0x%x", flags);
+  if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  std::vector<std::vector<int32_t>> tb;
+  std::vector<int32_t> sb, sn;
+  int64_t n_slots = 0;
+  akv_status s = plan_for_decode(B, tiers, n_tiers, split_tokens, tb, sb, sn, &n_slots);
+  if (s != AKV_OK) return s;
+  if (B == 0) return ok();
+  const HostLayout lay = host_layout(B, Hq, d, n_slots);
+  if (!workspace || !aligned(workspace, 256)) return fail(AKV_ERR_INVALID, "workspace must be 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    return fail(AKV_ERR_BUDGET, "workspace of %zu bytes, %zu needed", workspace_bytes, lay.total);
+  const size_t q_bytes = (size_t)B * Hq * d * 2, o_bytes = (size_t)B * Hq * d * sizeof(float),
+               l_bytes = (size_t)B * Hq * sizeof(float);
+  const HostArray hq = host_array(q_host, q_bytes), ho = host_array(o_host, o_bytes), hl = host_array(lse_host, l_bytes);
+  if (!hq.pinned || !ho.pinned || !hl.pinned)
+    return fail(AKV_ERR_NOT_PINNED, "q_host, o_host and lse_host must be page-locked host memory");
+  if (!aligned(q_host, 16) || !aligned(o_host, 4) || !aligned(lse_host, 4))
+    return fail(AKV_ERR_INVALID, "q_host must be 16-byte aligned, o_host and lse_host 4-byte aligned");
+  // the GPU touches host memory itself only where the driver vouches for the whole array
+  const bool kernel_in = !(flags & AKV_HOST_COPY_ENGINE) && hq.whole && aligned(hq.dev, 16);
+  const bool kernel_out = !(flags & AKV_HOST_COPY_ENGINE) && ho.whole && hl.whole;
+  std::vector<akv_tier> planned(tiers, tiers + n_tiers);
+  for (int i = 0; i < n_tiers; ++i) planned[i].slot_base = tb[i].data();
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* q_dev = ws + lay.q;
+  float* lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
+  float* o_part = reinterpret_cast<float*>(ws + lay.o_part);
+  const akv::CopyIn copy{kernel_in ? hq.dev : q_host, q_dev, q_bytes, kernel_in};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = akv::attend_impl(q_dev, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
+                       n_slots, variant, err_word, st, nullptr, &copy);
+  if (s != AKV_OK) return s;
+  float* o_dst = kernel_out ? static_cast<float*>(ho.dev) : reinterpret_cast<float*>(ws + lay.o);
+  float* l_dst = kernel_out ? static_cast<float*>(hl.dev) : reinterpret_cast<float*>(ws + lay.lse);
+  s = akv_merge_lse(o_part, lse_part, n_slots, sb.data(), sn.data(), B, Hq, d, o_dst, l_dst, stream);
+  if (s != AKV_OK || kernel_out) return s;
+  cudaError_t e = cudaMemcpyAsync(o_host, o_dst, o_bytes, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, l_dst, l_bytes, cudaMemcpyDeviceToHost, st);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "output copy");
 }
 
 }  // extern "C"

@@ -43,6 +43,15 @@ class DecodeStep:
         self.ws_bytes = akv.akv_decode_workspace_size(B, Hq, Hkv, d, self.tiers_c, split_tokens)
         self.workspace = torch.zeros(max(256, self.ws_bytes), dtype=torch.uint8, device=device)
 
+    def decode_host(self, q_host, o_host, lse_host, flags=0, variant=akv.AKV_VARIANT_AUTO, stream=None):
+        """The whole step with the query and the results in page-locked host memory."""
+        if getattr(self, "host_ws", None) is None:
+            self.host_ws_bytes = akv.akv_decode_host_workspace_size(self.B, self.Hq, self.Hkv, self.d, self.tiers_c,
+                                                                    self.split_tokens)
+            self.host_ws = torch.empty(max(256, self.host_ws_bytes), dtype=torch.uint8, device=self.o.device)
+        akv.akv_decode_host(q_host, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers_c, self.split_tokens,
+                            self.host_ws, self.host_ws_bytes, o_host, lse_host, flags, variant, self.err, stream)
+
     def decode(self, q, variant=akv.AKV_VARIANT_AUTO, stream=None):
         """The whole step in one call (split attention with the merge fused in)."""
         akv.akv_decode(q, self.B, self.Hq, self.Hkv, self.d, self.scale, self.tiers_c, self.split_tokens, self.workspace,

@@ -174,6 +174,36 @@ def test_append_tokens_refusals(akv):
     assert akv.lib.akv_append_tokens(ctypes.byref(t.c()), None, 1, 8, 128, None, None, None, None) == akv.AKV_ERR_INVALID
 
 
+def test_decode_host_refusals(akv):
+    """akv_decode_host checks its workspace, its flags and its host arrays before any launch;
+    arrays that are not page-locked (here plain numpy memory) are AKV_ERR_NOT_PINNED."""
+    t = _tier(akv, lens=[64])
+    B, Hq, Hkv, d = 1, 8, 2, 128
+    need = akv.akv_decode_host_workspace_size(B, Hq, Hkv, d, [t], 16)
+    up = lambda x: -(-x // 256) * 256
+    slots = 64 // 16
+    assert need == up(B * Hq * d * 2) + up(B * Hq * d * 4) + up(B * Hq * 4) + up(slots * Hq * 4) + up(slots * Hq * d * 4)
+    q = np.zeros((B, Hq, d), np.uint16)
+    o = np.zeros((B, Hq, d), np.float32)
+    lse = np.zeros((B, Hq), np.float32)
+    ws = 0x100000
+
+    def call(**kw):
+        a = dict(q=q, d=d, ws=ws, ws_bytes=need, flags=0)
+        a.update(kw)
+        with pytest.raises(akv.AkvError) as e:
+            akv.akv_decode_host(a["q"], B, Hq, Hkv, a["d"], 0.1, [t], 16, a["ws"], a["ws_bytes"], o, lse, a["flags"])
+        assert akv.lib.akv_last_error()
+        return e.value.status
+
+    assert call(flags=2) == akv.AKV_ERR_INVALID
+    assert call(d=96) == akv.AKV_ERR_UNSUPPORTED
+    assert call(ws=0x100010) == akv.AKV_ERR_INVALID
+    assert call(ws_bytes=need - 256) == akv.AKV_ERR_BUDGET
+    assert call() == akv.AKV_ERR_NOT_PINNED
+    akv.akv_decode_host(q, 0, Hq, Hkv, d, 0.1, [_tier(akv, lens=[])], 16, ws, need, o, lse)  # B = 0: nothing
+
+
 def test_header_is_plain_c():
     """include/akv.h is a C header: it compiles as C11 with strict warnings."""
     import shutil

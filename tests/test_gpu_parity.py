@@ -534,3 +534,35 @@ def test_hybrid_step_replays_from_cuda_graph(akv, wlmod, cuda, G, d):
         for a, b in zip(ref, outs):
             assert torch.equal(a.view(torch.int32), b.view(torch.int32))
     del g
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+@pytest.mark.parametrize("which", ["hybrid", "exact", "ragged"])
+def test_decode_host_matches_device_step(akv, wlmod, cuda, which, flags):
+    """akv_decode_host with the query and the results in page-locked host memory (flags 0:
+    the GPU reads and writes the host arrays itself; AKV_HOST_COPY_ENGINE: copy-engine
+    transfers) gives the bits of the device-memory step (akv_decode_attend + akv_merge_lse);
+    two calls in a row with alternating output buffers agree."""
+    import torch
+    if which == "hybrid":
+        w = wlmod.HybridResident(synth.WORKLOADS["hybrid"], cuda)
+    elif which == "exact":
+        w = wlmod.ExactResident(synth.WORKLOADS["exact"], cuda, B=3, T=3000)
+    else:
+        wl = synth.Workload("ragged-host", B=5, Hq=32, Hkv=8, d=128, split_tokens=512,
+                            extra={"window": 1024, "nu": 3.0})
+        w = wlmod.RaggedPaged(wl, cuda, lens=np.array([700, 1024, 3000, 17, 4100], np.int32))
+    step = w.step
+    step.step(w.q)
+    torch.cuda.synchronize()
+    ref_o, ref_lse = step.o.cpu(), step.lse.cpu()
+    q_host = torch.from_numpy(w.q_bits.view(np.int16)).pin_memory()
+    outs = [(torch.full(step.o.shape, float("nan")).pin_memory(), torch.full(step.lse.shape, float("nan")).pin_memory())
+            for _ in range(2)]
+    for o_h, l_h in outs:
+        step.decode_host(q_host, o_h, l_h, flags)
+    torch.cuda.synchronize()
+    assert int(step.err.item()) == 0
+    for o_h, l_h in outs:
+        assert torch.equal(o_h.view(torch.int32), ref_o.view(torch.int32))
+        assert torch.equal(l_h.view(torch.int32), ref_lse.view(torch.int32))
