@@ -47,8 +47,8 @@ def parse():
                     help="untimed steady-state run before the timed region (clocks settle, samples taken)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fuse", action="store_true",
-                    help="the fused decode call (merge folded into the attention launches) instead of separate "
-                         "attention and merge launches")
+                    help="time the one-call akv_decode (the library plans the slots and enqueues the attention "
+                         "and merge launches) instead of akv_decode_attend and akv_merge_lse calls")
     return ap.parse_args()
 
 
@@ -374,8 +374,8 @@ def run_ours(args):
             flush.fill_(1)
         run_step(w.q)
 
-    # attention launches (one per non-empty tier, B <= 256), plus the merge unless fused
-    launches_per_step = sum(1 for t in step.tiers if int(sum(t.lens)) > 0) + (0 if fuse else 1)
+    # attention launches (one per non-empty tier, B <= 256), plus the merge
+    launches_per_step = sum(1 for t in step.tiers if int(sum(t.lens)) > 0) + 1
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -524,7 +524,7 @@ def run_ours(args):
         dom_ms, dom_bytes = attend_avg_ms, kv_bytes
         dom_kernel = kernel_names[0] if len(live) == 1 else "attention launches"
         if fuse:
-            dom_kernel += " (merge fused in)"
+            dom_kernel += " + merge (one akv_decode call)"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = None if fuse else recorded_traffic(args.workload, dom_kernel)
     clocks = sampler.summary(t_soak, t_wall1 + 0.3)
@@ -534,7 +534,7 @@ def run_ours(args):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(describe(args.workload, wl, w), parallelism=f"independent replicas x{world}",
                                accumulate="f32", variant=args.variant,
-                               step="fused decode call (attention + merge)" if fuse
+                               step="one akv_decode call (attention launches + merge launch)" if fuse
                                else "attention launches + merge launch"),
                 "hbm_gbs": kv_bytes * world * args.steps / (ms * 1e-3) / 1e9,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -239,18 +239,14 @@ akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_s
  * the exact log-sum-exp merge ("Context beyond VRAM", "What I built": recent context
  * exact, older history compact, the two merged with exact attention arithmetic).
  *
- * The result equals akv_decode_attend followed by akv_merge_lse with the akv_plan_slots
- * layout (up to float32 rounding of the merge order), without a separate merge launch:
- * every finished split bumps a per-(sequence, KV head) counter and the split that
- * completes a sequence merges its query heads from the L2-resident partials.  Tiers'
- * slot_base arrays are ignored (the call plans its own slots).
+ * The call plans the akv_plan_slots layout itself (the tiers' slot_base arrays are ignored)
+ * and enqueues the launches of akv_decode_attend and akv_merge_lse, so the result is theirs
+ * bit for bit; the merge launch overlaps the attention launches' tail.
  *
  * workspace: caller-owned device scratch of at least akv_decode_workspace_size() bytes,
- * 256-byte aligned, holding the counters, then the LSE and O partials.  Zero it once after
- * allocating it; every call leaves the counters at zero again.  Calls that share a
- * workspace must not overlap on the device.  o, lse: device float32 [B][Hq][d], [B][Hq].
- * A smaller workspace gives AKV_ERR_BUDGET.  variant AKV_VARIANT_SIMT runs the CUDA-core
- * attention and the separate merge.
+ * 256-byte aligned, holding the LSE and then the O partials; its contents need no
+ * initialisation.  Calls that share a workspace must not overlap on the device.  o, lse:
+ * device float32 [B][Hq][d], [B][Hq].  A smaller workspace gives AKV_ERR_BUDGET.
  * ------------------------------------------------------------------------------------ */
 akv_status akv_decode_workspace_size(int B, int Hq, int Hkv, int d, const akv_tier* tiers, int n_tiers,
                                      int split_tokens, size_t* bytes);
@@ -303,9 +299,8 @@ akv_status akv_decode_host(const void* q_host, int B, int Hq, int Hkv, int d, fl
  * (see akv_decode_workspace_size), or with more than AKV_DECODE_STATIC_MAX_SEQ sequences
  * or 8 tiers, returns AKV_ERR_BUDGET / AKV_ERR_UNSUPPORTED and launches nothing.  The
  * first call on each device looks up the array's device address while that device is
- * current, so make it before any stream capture.  Every call shares the array: the
- * completion counters are cleared at the start of each call, everything else keeps the
- * last call's values, and calls whose work overlaps on the GPU race -- order them.
+ * current, so make it before any stream capture.  Every call shares the array: it keeps
+ * the last call's values, and calls whose work overlaps on the GPU race -- order them.
  * Arguments and results are those of akv_decode.
  * ------------------------------------------------------------------------------------ */
 #define AKV_DECODE_STATIC_MAX_BYTES (8u << 20)

@@ -45,9 +45,6 @@ struct SeqTable {
   int32_t item_base[kMaxSeqPerLaunch + 1];
   int32_t len[kMaxSeqPerLaunch];
   int32_t slot_base[kMaxSeqPerLaunch];
-  // fused decode: the sequence's slots over all tiers (merged by the item that completes them)
-  int32_t seq_slot_base[kMaxSeqPerLaunch];
-  int32_t seq_n_slots[kMaxSeqPerLaunch];
 };
 
 struct AttendParams {
@@ -61,11 +58,6 @@ struct AttendParams {
   int32_t Hq, Hkv, split_tokens;
   float scale_log2;      // softmax_scale * log2(e): scores are kept in base-2 units
   uint16_t centroids[16];
-  // fused decode: the item that completes a (sequence, KV head) also merges it into o / lse
-  int32_t fused;
-  int32_t* counters;     // [B][Hkv] finished splits; every merge resets its counter to 0
-  float* o;              // [B][Hq][D]
-  float* lse;            // [B][Hq]
   SeqTable seq;
 };
 
@@ -257,27 +249,18 @@ struct CopyIn {
   bool kernel;
 };
 
-// Fused decode: where the partials are merged.
-struct FusedArgs {
-  int32_t* counters;
-  float* o;
-  float* lse;
-  const int32_t* seq_slot_base;  // host [B]
-  const int32_t* seq_n_slots;    // host [B]
-};
-
-// Byte layout of a fused-decode workspace: counters [B][Hkv] int32, LSE partials
-// [n_slots][Hq] float, O partials [n_slots][Hq][d] float, each 256-byte aligned.
+// Byte layout of an akv_decode workspace: LSE partials [n_slots][Hq] float, then O partials
+// [n_slots][Hq][d] float, each 256-byte aligned.
 struct WorkspaceLayout {
-  size_t counters, lse, o, total;
+  size_t lse, o, total;
 };
 WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots);
 
-// Validated split attention of every tier (fused != null: merge folded in).
+// Validated split attention of every tier; copy_in (may be null) is enqueued after the checks
+// and before the first attention launch.
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused,
-                       const CopyIn* copy_in = nullptr);
+                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in = nullptr);
 
 // Set the thread's last-error message; returns st.
 akv_status set_error(akv_status st, const char* msg);

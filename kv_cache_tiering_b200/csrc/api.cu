@@ -103,8 +103,7 @@ akv::TierDev tier_dev(const akv_tier* t) {
 // Fill st for sequences [b0, b0 + n): sequence b owns ceil(len / unit) * mult work
 // items; returns the total.
 int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, const int32_t* slot_base,
-                       int unit, int mult = 1, const int32_t* seq_slot_base = nullptr,
-                       const int32_t* seq_n_slots = nullptr) {
+                       int unit, int mult = 1) {
   st.n_seq = n;
   st.b0 = b0;
   int64_t items = 0;
@@ -112,16 +111,12 @@ int64_t fill_seq_table(akv::SeqTable& st, int b0, int n, const int32_t* lens, co
     st.item_base[i] = (int32_t)items;
     st.len[i] = lens[b0 + i];
     st.slot_base[i] = slot_base ? slot_base[b0 + i] : 0;
-    st.seq_slot_base[i] = seq_slot_base ? seq_slot_base[b0 + i] : 0;
-    st.seq_n_slots[i] = seq_n_slots ? seq_n_slots[b0 + i] : 0;
     items += ceil_div(lens[b0 + i], unit) * mult;
   }
   st.item_base[n] = (int32_t)items;
   for (int i = n; i < akv::kMaxSeqPerLaunch; ++i) {
     st.len[i] = 0;
     st.slot_base[i] = 0;
-    st.seq_slot_base[i] = 0;
-    st.seq_n_slots[i] = 0;
     st.item_base[i + 1] = (int32_t)items;
   }
   return items;
@@ -134,8 +129,7 @@ namespace akv {
 WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   WorkspaceLayout l;
-  l.counters = 0;
-  l.lse = up((size_t)B * Hkv * sizeof(int32_t));
+  l.lse = 0;
   l.o = l.lse + up((size_t)n_slots * Hq * sizeof(float));
   l.total = l.o + up((size_t)n_slots * Hq * d * sizeof(float));
   return l;
@@ -461,7 +455,7 @@ namespace akv {
 
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const FusedArgs* fused, const CopyIn* copy_in) {
+                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in) {
   if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(AKV_ERR_INVALID, "Hq must be a positive multiple of Hkv");
   const int G = Hq / Hkv;
@@ -496,10 +490,6 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
   p.split_tokens = split_tokens;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   std::memcpy(p.centroids, akv::centroid_table_f16(), sizeof(p.centroids));
-  p.fused = (fused && variant != AKV_VARIANT_SIMT) ? 1 : 0;
-  p.counters = fused ? fused->counters : nullptr;
-  p.o = fused ? fused->o : nullptr;
-  p.lse = fused ? fused->lse : nullptr;
   // Every launch is checked (and every refusal made) before the first one is enqueued.  The
   // first two launches are kept: that is all the side-by-side case needs, and a call with
   // more launches rebuilds each one's parameters while enqueuing, so no call allocates.
@@ -515,8 +505,7 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
         // the CUDA-core kernels take a (split, KV head) grid; the tensor-core kernels a flat
         // list of (split, KV head) items
         const int64_t items =
-            fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv,
-                           fused ? fused->seq_slot_base : nullptr, fused ? fused->seq_n_slots : nullptr);
+            fill_seq_table(p.seq, b0, n, tiers[i].lens, tiers[i].slot_base, split_tokens, simt ? 1 : Hkv);
         if (items == 0) continue;
         if (items > INT32_MAX) return fail(AKV_ERR_UNSUPPORTED, "too many splits in one launch");
         int64_t max_len = 0;
@@ -575,7 +564,7 @@ akv_status akv_decode_attend(const void* q, int B, int Hq, int Hkv, int d, float
                              const akv_tier* tiers, int n_tiers, int split_tokens, float* o_part, float* lse_part,
                              int64_t n_slots, int variant, int32_t* err_word, akv_stream_t stream) {
   return akv::attend_impl(q, B, Hq, Hkv, d, softmax_scale, tiers, n_tiers, split_tokens, o_part, lse_part, n_slots,
-                     variant, err_word, reinterpret_cast<cudaStream_t>(stream), nullptr);
+                     variant, err_word, reinterpret_cast<cudaStream_t>(stream));
 }
 
 akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_slots, const int32_t* seq_slot_base,
@@ -617,7 +606,7 @@ akv_status akv_merge_lse(const float* o_part, const float* lse_part, int64_t n_s
   return ok();
 }
 
-// Plan the standard slot layout for a fused decode (host vectors).
+// Plan the standard slot layout for a whole decode step (host vectors).
 static akv_status plan_for_decode(int B, const akv_tier* tiers, int n_tiers, int split_tokens,
                                   std::vector<std::vector<int32_t>>& tier_base, std::vector<int32_t>& seq_base,
                                   std::vector<int32_t>& seq_n, int64_t* n_slots) {
@@ -671,16 +660,11 @@ akv_status akv_decode(const void* q, int B, int Hq, int Hkv, int d, float softma
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* lse_part = reinterpret_cast<float*>(ws + lay.lse);
   float* o_part = reinterpret_cast<float*>(ws + lay.o);
-  akv::FusedArgs fa{reinterpret_cast<int32_t*>(ws + lay.counters), o, lse, sb.data(), sn.data()};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   s = akv::attend_impl(q, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
-                  n_slots, variant, err_word, st, &fa);
+                  n_slots, variant, err_word, st);
   if (s != AKV_OK) return s;
-  // the CUDA-core path, and sequences without any token, take the separate merge
-  bool need_merge = variant == AKV_VARIANT_SIMT;
-  for (int b = 0; b < B && !need_merge; ++b) need_merge = sn[b] == 0;
-  if (need_merge) return akv_merge_lse(o_part, lse_part, n_slots, sb.data(), sn.data(), B, Hq, d, o, lse, stream);
-  return ok();
+  return akv_merge_lse(o_part, lse_part, n_slots, sb.data(), sn.data(), B, Hq, d, o, lse, stream);
 }
 
 }  // extern "C"
@@ -788,7 +772,7 @@ akv_status akv_decode_host(const void* q_host, int B, int Hq, int Hkv, int d, fl
   const akv::CopyIn copy{kernel_in ? hq.dev : q_host, q_dev, q_bytes, kernel_in};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   s = akv::attend_impl(q_dev, B, Hq, Hkv, d, softmax_scale, planned.data(), n_tiers, split_tokens, o_part, lse_part,
-                       n_slots, variant, err_word, st, nullptr, &copy);
+                       n_slots, variant, err_word, st, &copy);
   if (s != AKV_OK) return s;
   float* o_dst = kernel_out ? static_cast<float*>(ho.dev) : reinterpret_cast<float*>(ws + lay.o);
   float* l_dst = kernel_out ? static_cast<float*>(hl.dev) : reinterpret_cast<float*>(ws + lay.lse);

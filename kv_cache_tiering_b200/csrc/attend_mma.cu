@@ -413,106 +413,6 @@ __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it
 }
 
 // ------------------------------------------------------------------------------------
-// fused decode: the item that completes a (sequence, KV head) merges its query heads
-// ------------------------------------------------------------------------------------
-// Every finished item fences its partial writes and bumps the (sequence, KV head) counter;
-// the item that brings it to the sequence's slot count merges slots seq_slot_base ..
-// + seq_n_slots - 1 in slot order (max, exp weights, weighted sum -- the LSE merge) and
-// resets the counter.  Partials of other CTAs are read past L1.
-template <int D, int G>
-__device__ __forceinline__ void merge_tail(const AttendParams& p, const Item& it, int t, int nthreads) {
-  const int base = p.seq.seq_slot_base[it.bl], n = p.seq.seq_n_slots[it.bl];
-  for (int i = t; i < G * D; i += nthreads) {
-    const int h = i / D, dim = i % D, hq = it.kvh * G + h;
-    float M = -INFINITY;
-    for (int s = 0; s < n; ++s) M = fmaxf(M, __ldcg(p.lse_part + (size_t)(base + s) * p.Hq + hq));
-    float o = 0.f, L = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-      for (int s = 0; s < n; ++s) {
-        const float w = expf(__ldcg(p.lse_part + (size_t)(base + s) * p.Hq + hq) - M);
-        L += w;
-        o = fmaf(w, __ldcg(p.o_part + ((size_t)(base + s) * p.Hq + hq) * D + dim), o);
-      }
-      o /= L;
-    }
-    p.o[((size_t)it.b * p.Hq + hq) * D + dim] = o;
-    if (dim == 0) p.lse[(size_t)it.b * p.Hq + hq] = (M == -INFINITY) ? -INFINITY : M + logf(L);
-  }
-}
-
-// The same merge by a whole CTA of NT threads, through shared memory `sm` (at least
-// 2 G + max(NT, G kTailChunk) floats; every thread of the CTA calls it).  Pass 1 finds each head's
-// maximum LSE over the sequence's slots; pass 2 takes the slots in chunks: their weights
-// exp(lse - M) go to shared memory, then every thread accumulates its outputs over the
-// chunk with independent loads.  Same formula and slot order as merge_tail.
-constexpr int kTailChunk = 64;
-template <int D, int G, int NT>
-__device__ void merge_tail_cta(const AttendParams& p, const Item& it, float* sm) {
-  static_assert(NT % G == 0, "thread layout of the tail");
-  constexpr int E = (G * D + NT - 1) / NT;  // outputs per thread (the last ones may be past G D)
-  const int t = threadIdx.x;
-  const int base = p.seq.seq_slot_base[it.bl], n = p.seq.seq_n_slots[it.bl];
-  const float* lse_p = p.lse_part + (size_t)base * p.Hq + it.kvh * G;
-  float* Mh = sm;             // [G]
-  float* Lh = sm + G;         // [G]
-  float* wsm = sm + 2 * G;    // [kTailChunk][G]
-  // pass 1: maxima (thread t takes head t % G, slots t / G, t / G + NT / G, ...)
-  float m = -INFINITY;
-  for (int s = t / G; s < n; s += NT / G) m = fmaxf(m, __ldcg(lse_p + (size_t)s * p.Hq + t % G));
-  wsm[t] = m;
-  __syncthreads();
-  if (t < G) {
-    float M = -INFINITY;
-    for (int k = t; k < NT; k += G) M = fmaxf(M, wsm[k]);
-    Mh[t] = M;
-  }
-  __syncthreads();
-  // pass 2: weights per chunk, then the weighted sums
-  float o[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) o[e] = 0.f;
-  float L = 0.f;
-  for (int c0 = 0; c0 < n; c0 += kTailChunk) {
-    const int nc = min(kTailChunk, n - c0);
-    for (int k = t; k < nc * G; k += NT) {
-      const int h = k % G;
-      wsm[k] = Mh[h] == -INFINITY ? 0.f : expf(__ldcg(lse_p + (size_t)(c0 + k / G) * p.Hq + h) - Mh[h]);
-    }
-    __syncthreads();
-    if (t < G)
-      for (int s = 0; s < nc; ++s) L += wsm[s * G + t];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int i = t + e * NT, h = i / D, dim = i % D;
-      if (i >= G * D) break;
-      const float* op = p.o_part + ((size_t)(base + c0) * p.Hq + it.kvh * G + h) * D + dim;
-      float a = o[e];
-#pragma unroll 8
-      for (int s = 0; s < nc; ++s) a = fmaf(wsm[s * G + h], __ldcg(op + (size_t)s * p.Hq * D), a);
-      o[e] = a;
-    }
-    __syncthreads();
-  }
-  if (t < G) Lh[t] = L;
-  __syncthreads();
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = t + e * NT, h = i / D, dim = i % D, hq = it.kvh * G + h;
-    if (i >= G * D) break;
-    const float M = Mh[h];
-    p.o[((size_t)it.b * p.Hq + hq) * D + dim] = M == -INFINITY ? 0.f : o[e] / Lh[h];
-    if (dim == 0) p.lse[(size_t)it.b * p.Hq + hq] = M == -INFINITY ? -INFINITY : M + logf(Lh[h]);
-  }
-}
-
-// Count a finished item; true for the caller that completed the (sequence, KV head).
-__device__ __forceinline__ bool finish_item(const AttendParams& p, const Item& it) {
-  const int old = atomicAdd(p.counters + (size_t)it.b * p.Hkv + it.kvh, 1);
-  return old + 1 == p.seq.seq_n_slots[it.bl];
-}
-
-// ------------------------------------------------------------------------------------
 // exact BF16 tier
 // ------------------------------------------------------------------------------------
 template <int D, int G, int NW, int NST>
@@ -525,8 +425,7 @@ struct Bf16Cfg {
   static constexpr int AREA = NW * G * D;          // floats
   static constexpr int FLOATS = AREA + 3 * NW * G;  // area, m, l, factors
   static constexpr int BAR_OFF = RINGS + FLOATS * 4;
-  static constexpr int FLAG_OFF = BAR_OFF + NW * NST * 8;
-  static constexpr size_t SMEM = FLAG_OFF + 16 + 1024;  // + alignment slack
+  static constexpr size_t SMEM = BAR_OFF + NW * NST * 8 + 1024;  // + alignment slack
 };
 
 // Byte offset, inside a TMA-swizzled tile, of 16-byte chunk c (of D/8) of row r.
@@ -705,18 +604,6 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
     chain_to_smem<D, G>(acc, m_run, l_run, area + w * G * D, mws + w * G, lws + w * G, dim_of);
     group_sync<NW>(gi);
     merge_item<D, G, NW, false>(p, it, gi, area, mws, lws, fac, nullptr);
-    if (p.fused) {
-      int* flag = reinterpret_cast<int*>(smem + C::FLAG_OFF);
-      __threadfence();
-      group_sync<NW>(gi);
-      if (threadIdx.x == 0) *flag = finish_item(p, it) ? 1 : 0;
-      group_sync<NW>(gi);
-      if (*flag) {  // CTA-uniform
-        __threadfence();
-        merge_tail_cta<D, G, NW * 32>(p, it, area);
-        if (threadIdx.x == 0) p.counters[(size_t)it.b * p.Hkv + it.kvh] = 0;
-      }
-    }
     group_sync<NW>(gi);
   }
   if (!ok) {
@@ -1219,17 +1106,6 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
       } else {
         *reinterpret_cast<float2*>(dst) = make_float2(x[0], x[1]);
-      }
-    }
-    if (p.fused) {
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = finish_item(p, it) ? 1 : 0;
-      if (__shfl_sync(kFull, last, 0)) {
-        __threadfence();
-        merge_tail<D, G>(p, it, lane, 32);
-        if (lane == 0) p.counters[(size_t)it.b * p.Hkv + it.kvh] = 0;
       }
     }
     __syncwarp();

@@ -1,6 +1,6 @@
-// akv_decode_static: the fused decode step for callers that cannot allocate device memory.
+// akv_decode_static: the whole decode step for callers that cannot allocate device memory.
 //
-// akv_decode needs a scratch workspace for its split partials and completion counters,
+// akv_decode needs a scratch workspace for its split partials,
 // and leaves it to the caller to provide one.  Some callers have no way to get device
 // memory at the moment they decode: code running inside a host function enqueued on a
 // stream (where CUDA forbids API calls such as cudaMalloc), a plugin living in a process
@@ -14,9 +14,8 @@
 // array's name as a device address, so the first call on each device looks the address
 // up with cudaGetSymbolAddress while that device is current, and later calls on the
 // device reuse it; make that first call before any stream capture.  All calls share the
-// one array: it keeps whatever the last call left in it, the completion counters are
-// cleared at the start of every call, and two calls whose work overlaps on the GPU (two
-// streams, say) race on the array -- order them.
+// one array: it keeps whatever the last call left in it, and two calls whose work overlaps
+// on the GPU (two streams, say) race on the array -- order them.
 #include <mutex>
 
 #include "akv_internal.cuh"
@@ -90,17 +89,10 @@ extern "C" akv_status akv_decode_static(const void* q, int B, int Hq, int Hkv, i
   if ((s = scratch_address(&scratch)) != AKV_OK) return s;
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // counters must start at zero; whatever an earlier call left there is cleared
-  cudaError_t e = cudaMemsetAsync(ws + lay.counters, 0, (size_t)B * Hkv * sizeof(int32_t), st);
-  if (e != cudaSuccess) return akv::set_error(AKV_ERR_CUDA, cudaGetErrorString(e));
   float* lse_part = reinterpret_cast<float*>(ws + lay.lse);
   float* o_part = reinterpret_cast<float*>(ws + lay.o);
-  akv::FusedArgs fa{reinterpret_cast<int32_t*>(ws + lay.counters), o, lse, seq_base, seq_n};
   s = akv::attend_impl(q, B, Hq, Hkv, d, softmax_scale, planned, n_tiers, split_tokens, o_part, lse_part, n_slots,
-                       variant, err_word, st, &fa);
+                       variant, err_word, st);
   if (s != AKV_OK) return s;
-  bool need_merge = variant == AKV_VARIANT_SIMT;
-  for (int b = 0; b < B && !need_merge; ++b) need_merge = seq_n[b] == 0;
-  if (need_merge) return akv_merge_lse(o_part, lse_part, n_slots, seq_base, seq_n, B, Hq, d, o, lse, stream);
-  return AKV_OK;
+  return akv_merge_lse(o_part, lse_part, n_slots, seq_base, seq_n, B, Hq, d, o, lse, stream);
 }

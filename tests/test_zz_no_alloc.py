@@ -1,7 +1,7 @@
 """The allocation-free decode entry point, tested last.
 
 akv_decode_static is for callers that cannot allocate device memory at decode time: it
-runs the same fused decode as akv_decode on a fixed scratch array inside the library
+runs the same decode step as akv_decode on a fixed scratch array inside the library
 instead of a caller-provided workspace.  This test calls it through the C ABI twice in a
 row and checks each result against akv_decode on the same inputs; it also checks that a
 step too large for the fixed scratch is refused.  It must pass alone in a fresh process
