@@ -204,9 +204,10 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
  * a staged run equals the resident run bit for bit.  Page ids outside [0, n_pages) set
  * AKV_EFLAG_BOUNDS in *err_word (device, may be NULL) and read page 0 instead.
  * Streams: asynchronous on `stream`; work enqueued on `stream` after the call sees every
- * partial.  With one BF16 and one compact launch (tensor-core variants) the library may run
- * the BF16 launch on an internal stream of the current device, forked from and joined back
- * to `stream` with events, so the two grids share the SMs (same bits as launched in a row).
+ * partial.  With one BF16 and one compact launch (tensor-core variants) and `stream` on the
+ * current device, the library may run the BF16 launch on an internal stream of that device,
+ * forked from and joined back to `stream` with events, so the two grids share the SMs (same
+ * bits as launched in a row).
  * That internal stream serves every such call on the device: a call whose `stream` is being
  * captured into a graph must not run while another host thread enqueues such a call on the
  * same device.  The first such call on a device creates the stream and its two events; make

@@ -423,6 +423,16 @@ cudaError_t side_lane(SideLane*& out) {
 // same time.  The side stream starts after the work enqueued on `st` so far, and `st` resumes
 // after both launches; each split's arithmetic is independent of the grid, so the partials
 // are the same bits as from two launches in a row.
+// Whether `st` belongs to the current device (the side stream's device).
+bool stream_on_current_device(cudaStream_t st) {
+  int cur = 0, dev = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(st, &dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return cur == dev;
+}
+
 akv_status side_by_side(const PlannedLaunch& c, const PlannedLaunch& x, int share, int rest, int d, int G,
                         cudaStream_t st) {
   std::lock_guard<std::mutex> lock(side_mutex());
@@ -540,7 +550,7 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
     if (cs != AKV_OK) return cs;
   }
   const int sms = akv::sm_count();
-  if (!simt && n_launch == 2 && two[0].kind != two[1].kind && sms >= 2) {
+  if (!simt && n_launch == 2 && two[0].kind != two[1].kind && sms >= 2 && stream_on_current_device(st)) {
     const PlannedLaunch& c = two[0].kind == AKV_TIER_CODES4 ? two[0] : two[1];
     const PlannedLaunch& x = two[0].kind == AKV_TIER_CODES4 ? two[1] : two[0];
     const int share = compact_sm_share(sms, c.items, akv::codes_warps_per_cta(G), ceil_div(c.split_len, 16), x.items,
