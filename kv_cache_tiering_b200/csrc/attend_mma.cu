@@ -364,14 +364,12 @@ __device__ __forceinline__ void warp_fwht(float (&x)[P]) {
 }
 
 // Merge the NW chain states of a finished item (group threads) and write its partials.
-// First the G per-head statistics and the NW x G chain factors exp2(m_w - M) / L
-// (/ D as well in the rotated basis) are computed once; then every output is one dot
-// product over chains.  kRotate: the merged rows are in the rotated basis; rotate back.
-template <int D, int G, int NW, bool kRotate>
+// First the G per-head statistics and the NW x G chain factors exp2(m_w - M) / L are
+// computed once; then every output is one dot product over chains.
+template <int D, int G, int NW>
 __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it, int gi, float* area, float* mws,
-                                           float* lws, float* fac, float* stage) {
+                                           float* lws, float* fac) {
   const int tg = threadIdx.x - gi * NW * 32;  // thread index within the group
-  const int warp_in = tg >> 5, lane = threadIdx.x & 31;
   if (tg < G) {
     const int h = tg;
     float M = -INFINITY;
@@ -380,7 +378,7 @@ __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it
     float L = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) L = fmaf(lws[w * G + h], exp2f(mws[w * G + h] - M), L);
-    const float inv = 1.f / (kRotate ? (float)D * L : L);
+    const float inv = 1.f / L;
 #pragma unroll
     for (int w = 0; w < NW; ++w) fac[w * G + h] = exp2f(mws[w * G + h] - M) * inv;  // 0 for an empty chain
     p.lse_part[(size_t)it.slot * p.Hq + it.kvh * G + h] = kLn2 * (M + log2f(L));
@@ -391,24 +389,7 @@ __device__ __forceinline__ void merge_item(const AttendParams& p, const Item& it
     float o = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) o = fmaf(area[(w * G + h) * D + dim], fac[w * G + h], o);
-    if constexpr (kRotate) {
-      stage[i] = o;
-    } else {
-      p.o_part[((size_t)it.slot * p.Hq + it.kvh * G + h) * D + dim] = o;
-    }
-  }
-  if constexpr (kRotate) {
-    group_sync<NW>(gi);
-    constexpr int P = D / 32;
-    for (int h = warp_in; h < G; h += NW) {
-      float x[P];
-#pragma unroll
-      for (int j = 0; j < P; ++j) x[j] = stage[h * D + P * lane + j];
-      warp_fwht<P>(x);
-      float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
-#pragma unroll
-      for (int j = 0; j < P; ++j) dst[j] = x[j];
-    }
+    p.o_part[((size_t)it.slot * p.Hq + it.kvh * G + h) * D + dim] = o;
   }
 }
 
@@ -603,7 +584,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
     }
     chain_to_smem<D, G>(acc, m_run, l_run, area + w * G * D, mws + w * G, lws + w * G, dim_of);
     group_sync<NW>(gi);
-    merge_item<D, G, NW, false>(p, it, gi, area, mws, lws, fac, nullptr);
+    merge_item<D, G, NW>(p, it, gi, area, mws, lws, fac);
     group_sync<NW>(gi);
   }
   if (!ok) {
