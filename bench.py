@@ -172,7 +172,8 @@ def make_workload(name: str, device, rank: int):
     return wl, w, tokens
 
 
-def describe(name, wl, w):
+def describe(name, wl, w=None):
+    """The config of a bench line; w (the device workload) adds its bytes per step."""
     d = {"workload": {
         "exact": "exact-tier GQA decode: batch 8, 32 q / 8 KV heads, d 128, 8192 BF16 tokens, contiguous, 512-token splits",
         "tiny": "tiny exact decode: batch 1, 1 q / 1 KV head, d 64, 256 BF16 tokens, 4 splits of 64",
@@ -183,10 +184,11 @@ def describe(name, wl, w):
         "staged": "staged 128k history: batch 1, 16 layers, 32 q / 8 KV heads, d 128, 131072 BF16 tokens per layer "
                   "in pinned host memory, 4096-token chunks through a 2-buffer device region, one token appended "
                   "per step",
-    }[name], "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.d, "split_tokens": wl.split_tokens,
-        "kv_bytes_per_step": w.kv_bytes()}
-    d["l2"] = ("inputs larger than the 126 MB L2, no flush" if w.kv_bytes() > 126e6
-               else "L2 flushed (256 MB write) before every step")
+    }[name], "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.d, "split_tokens": wl.split_tokens}
+    if w is not None:
+        d["kv_bytes_per_step"] = w.kv_bytes()
+        d["l2"] = ("inputs larger than the 126 MB L2, no flush" if w.kv_bytes() > 126e6
+                   else "L2 flushed (256 MB write) before every step")
     return d
 
 
@@ -316,7 +318,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "reference": "float64 numpy oracle on the host CPU",
+            "config": {**describe(args.workload, wl), "reference": "float64 numpy oracle on the host CPU",
                        "step": desc},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{args.steps} units: {desc}"},
