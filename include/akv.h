@@ -210,8 +210,9 @@ akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, i
  * bits as launched in a row).
  * That internal stream serves every such call on the device: a call whose `stream` is being
  * captured into a graph must not run while another host thread enqueues such a call on the
- * same device.  The first such call on a device creates the stream and its two events; make
- * it before any capture.  Apart from an error message, no call allocates memory.
+ * same device, and a call captured into a graph must be made with the capturing stream's
+ * device current.  The first such call on a device creates the stream and its two events;
+ * make it before any capture.  Apart from an error message, no call allocates memory.
  * ------------------------------------------------------------------------------------ */
 enum { AKV_VARIANT_AUTO = 0, AKV_VARIANT_SIMT = 1, AKV_VARIANT_MMA = 2 };
 

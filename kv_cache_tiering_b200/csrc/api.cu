@@ -423,8 +423,16 @@ cudaError_t side_lane(SideLane*& out) {
 // same time.  The side stream starts after the work enqueued on `st` so far, and `st` resumes
 // after both launches; each split's arithmetic is independent of the grid, so the partials
 // are the same bits as from two launches in a row.
-// Whether `st` belongs to the current device (the side stream's device).
+// Whether `st` belongs to the current device (the side stream's device).  A stream being
+// captured into a graph is not asked (the query is not allowed during capture): the call
+// must then be made with the stream's device current, as every call on a stream must.
 bool stream_on_current_device(cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return true;
   int cur = 0, dev = 0;
   if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(st, &dev) != cudaSuccess) {
     cudaGetLastError();
