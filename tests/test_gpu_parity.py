@@ -564,3 +564,30 @@ def test_decode_host_matches_device_step(akv, wlmod, cuda, which, flags):
     for o_h, l_h in outs:
         assert torch.equal(o_h.view(torch.int32), ref_o.view(torch.int32))
         assert torch.equal(l_h.view(torch.int32), ref_lse.view(torch.int32))
+
+
+@pytest.mark.parametrize("variant", ["simt", "mma"])
+def test_hybrid_more_sequences_than_one_launch(akv, wlmod, cuda, variant):
+    """300 sequences: each tier takes two launches (256 sequences at most per launch), so a
+    step makes four attention launches.  Sampled sequences match the oracle, and
+    akv_decode_host (its query copy enqueued before the first of the four) gives the step's
+    bits."""
+    import torch
+    wl = synth.Workload("hybrid-many", B=300, Hq=8, Hkv=2, d=64, split_tokens=64, extra={"T": 150, "window": 50})
+    w = wlmod.HybridResident(wl, cuda)
+    step = w.step
+    step.step(w.q, variant_id(akv, variant))
+    torch.cuda.synchronize()
+    assert int(w.enc_err.item()) == 0 and int(step.err.item()) == 0
+    for b in (0, 1, 255, 256, 299):
+        (partials, merged, direct), _ = _oracle_hybrid(wl, w, b)
+        check_partials(step, 0, b, partials[0])
+        check_partials(step, 1, b, partials[1])
+        check_merged(step, b, direct)
+    q_host = torch.from_numpy(w.q_bits.view(np.int16)).pin_memory()
+    o_h = torch.full(step.o.shape, float("nan")).pin_memory()
+    l_h = torch.full(step.lse.shape, float("nan")).pin_memory()
+    step.decode_host(q_host, o_h, l_h, 0, variant_id(akv, variant))
+    torch.cuda.synchronize()
+    assert torch.equal(o_h.view(torch.int32), step.o.cpu().view(torch.int32))
+    assert torch.equal(l_h.view(torch.int32), step.lse.cpu().view(torch.int32))
