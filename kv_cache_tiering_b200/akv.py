@@ -251,11 +251,16 @@ def plan_slots(tier_lens, split_tokens: int):
     return bases, seq_base, seq_n, n.value
 
 
-def akv_append_tokens(tier: Tier, pos, B: int, Hkv: int, d: int, new_k, new_v, err_word=None, stream=None) -> None:
-    """Write row b of new_k / new_v ([B][Hkv][d] bf16, device) to token pos[b] of a BF16 tier."""
-    t = tier.c()
+def akv_append_tokens(tier, pos, B: int, Hkv: int, d: int, new_k, new_v, err_word=None, stream=None) -> None:
+    """Write row b of new_k / new_v ([B][Hkv][d] bf16, device) to token pos[b] of a BF16 tier
+    (a Tier, or a one-tier TierArray marshalled once)."""
+    if isinstance(tier, TierArray):
+        arg = tier.arr
+    else:
+        t = tier.c()
+        arg = ctypes.byref(t)
     p = _host_i32(pos)
-    _check(lib.akv_append_tokens(ctypes.byref(t), p.ctypes.data, B, Hkv, d, _ptr(new_k), _ptr(new_v), _ptr(err_word),
+    _check(lib.akv_append_tokens(arg, p.ctypes.data, B, Hkv, d, _ptr(new_k), _ptr(new_v), _ptr(err_word),
                                  _stream(stream)))
 
 

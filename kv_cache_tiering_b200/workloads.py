@@ -617,6 +617,23 @@ class AgingHybrid:
         self.steps_done = 0
         self.aged_blocks = 0
         self.encode_events = None  # a list: every aging encode is bracketed by timing events
+        # host arrays the marshalled tiers point to, updated in place every step: lengths, the
+        # append positions and the slot plan (replanned only when a tier's split count changes)
+        H = wl.Hkv
+        self._cp_len = np.zeros(self.B, np.int32)
+        self._ex_len = np.zeros(self.B, np.int32)
+        self._pos = np.zeros(self.B, np.int32)
+        self._cp_base = np.zeros(self.B, np.int32)
+        self._ex_base = np.zeros(self.B, np.int32)
+        self._seq_base = np.zeros(self.B, np.int32)
+        self._seq_n = np.zeros(self.B, np.int32)
+        self._n_slots = 0
+        self._plan_counts = None
+        codes = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=self._cp_len, slot_base=self._cp_base,
+                         paged=True, page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1],
+                         n_pages=self.n_cp, stride_seq=H, stride_head=1)
+        self._attend_tiers = akv.TierArray([codes, self._exact_tier(self._ex_len, self._ex_base)])
+        self._append_tier = akv.TierArray([self._exact_tier(self._ex_len)])
 
     def inputs(self, step: int):
         """Device q [B][Hq][d] and new K, V rows [B][Hkv][d] of decode step ``step``."""
@@ -640,7 +657,9 @@ class AgingHybrid:
         wl, H, d, B = self.wl, self.wl.Hkv, self.wl.d, self.B
         dev = self.device
         # 1. append: token win[b] of the window, through the window's page table
-        akv.akv_append_tokens(self._exact_tier(), self.win.astype(np.int32), B, H, d, k_new, v_new, self.err, stream)
+        self._ex_len[:] = self.win
+        self._pos[:] = self.win
+        akv.akv_append_tokens(self._append_tier, self._pos, B, H, d, k_new, v_new, self.err, stream)
         self.win += 1
         # 2. age: a window of W + 16 tokens hands its oldest page to the compact tier
         aging = [b for b in range(B) if self.win[b] >= self.W + 16]
@@ -681,14 +700,17 @@ class AgingHybrid:
                 self._tables_done.record(cur)
             self.aged_blocks += n
         # 3. attend both tiers into their planned slots, then merge
-        cp_len, ex_len = self.c.astype(np.int32), self.win.astype(np.int32)
-        bases, seq_base, seq_n, n_slots = akv.plan_slots([cp_len, ex_len], wl.split_tokens)
-        codes = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=cp_len, slot_base=bases[0], paged=True,
-                         page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1], n_pages=self.n_cp,
-                         stride_seq=H, stride_head=1)
-        exact = self._exact_tier(ex_len, bases[1])
-        akv.akv_decode_attend(q, B, wl.Hq, H, d, wl.scale, [codes, exact], wl.split_tokens, self.o_part,
-                              self.lse_part, n_slots, variant, self.err, stream)
-        akv.akv_merge_lse(self.o_part, self.lse_part, n_slots, seq_base, seq_n, B, wl.Hq, d, self.o, self.lse,
-                          stream)
+        self._cp_len[:] = self.c
+        self._ex_len[:] = self.win
+        split = wl.split_tokens
+        counts = ((self._cp_len + split - 1) // split, (self._ex_len + split - 1) // split)
+        if self._plan_counts is None or any(not np.array_equal(a, b) for a, b in zip(counts, self._plan_counts)):
+            bases, seq_base, seq_n, self._n_slots = akv.plan_slots([self._cp_len, self._ex_len], split)
+            self._cp_base[:], self._ex_base[:] = bases[0], bases[1]
+            self._seq_base[:], self._seq_n[:] = seq_base, seq_n
+            self._plan_counts = counts
+        akv.akv_decode_attend(q, B, wl.Hq, H, d, wl.scale, self._attend_tiers, split, self.o_part, self.lse_part,
+                              self._n_slots, variant, self.err, stream)
+        akv.akv_merge_lse(self.o_part, self.lse_part, self._n_slots, self._seq_base, self._seq_n, B, wl.Hq, d, self.o,
+                          self.lse, stream)
         self.steps_done += 1
