@@ -188,7 +188,7 @@ def describe(name, wl, w=None):
     if w is not None:
         d["kv_bytes_per_step"] = w.kv_bytes()
         d["l2"] = ("inputs larger than the 126 MB L2, no flush" if w.kv_bytes() > 126e6
-                   else "L2 flushed (256 MB write) before every step")
+                   else "L2 flushed (256 MB write) before every step; each step timed by its own events, the flush not timed")
     return d
 
 
@@ -405,10 +405,15 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.monotonic()
+    # with an L2 flush between steps (inputs smaller than L2), each step is bracketed by its own
+    # events after the flush, and the time is the sum of the steps: the flush is not timed
+    step_ev = ([(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)] if flush is not None else None)
     start.record(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(1)
+            step_ev[i][0].record(stream)
         k = i // SAMPLE if i % SAMPLE == 0 else -1
         if k >= 0:
             a0[k].record(stream)
@@ -424,12 +429,14 @@ def run_ours(args):
             a1[k].record(stream)
         if not fuse:
             step.merge(stream)
+        if flush is not None:
+            step_ev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.monotonic()
     if dist:
         dist.barrier()
-    ms = start.elapsed_time(end)
+    ms = start.elapsed_time(end) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
     attend_ms = [a0[k].elapsed_time(a1[k]) for k in range(len(sampled))]
     tier_ms = ([statistics.fmean(bounds[j][k].elapsed_time(bounds[j + 1][k]) for k in range(len(sampled)))
                 for j in range(len(live))] if per_tier else None)
@@ -459,11 +466,17 @@ def run_ours(args):
     ev_used = [torch.cuda.Event() for _ in range(2)]  # step j's compute is done with its buffers
     ev_out = [torch.cuda.Event() for _ in range(2)]   # download j landed
 
+    e2e_ev = None  # per-step events when the L2 flush sits between steps (set for the timed run)
+
     def e2e_host_step(i):
         j = i % 2
         if flush is not None:
             flush.fill_(1)
+            if e2e_ev is not None:
+                e2e_ev[i][0].record(stream)
         step.decode_host(q_host, o_host[j], lse_host[j], 0, variant, stream)
+        if flush is not None and e2e_ev is not None:
+            e2e_ev[i][1].record(stream)
 
     def e2e_copy_step(i):
         j, st_j = i % 2, pair[i % 2]
@@ -491,6 +504,9 @@ def run_ours(args):
         e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if flush is not None and not fuse:
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
     if dist:
         dist.barrier()
     e0.record(stream)
@@ -502,7 +518,7 @@ def run_ours(args):
         stream.wait_event(ev_out[args.steps % 2])
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e0.elapsed_time(e1) if e2e_ev is None else sum(a.elapsed_time(b) for a, b in e2e_ev)
     if dist:
         e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     sampler.stop()
