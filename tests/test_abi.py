@@ -174,6 +174,18 @@ def test_append_tokens_refusals(akv):
     assert akv.lib.akv_append_tokens(ctypes.byref(t.c()), None, 1, 8, 128, None, None, None, None) == akv.AKV_ERR_INVALID
 
 
+def test_decode_workspace_size_is_the_documented_layout(akv):
+    """akv_decode's workspace holds the LSE partials, then the O partials, each rounded up to
+    256 bytes; the slots are the akv_plan_slots layout of the tiers."""
+    up = lambda x: -(-x // 256) * 256
+    tiers = [_tier(akv, lens=[100, 0, 1024]), _tier(akv, kind=akv.AKV_TIER_CODES4, lens=[30, 5, 0],
+                                                      stride_head=2, stride_token=1)]
+    _, _, _, n_slots = akv.plan_slots([[100, 0, 1024], [30, 5, 0]], 64)
+    for Hq, Hkv, d in ((8, 2, 128), (32, 8, 64)):
+        got = akv.akv_decode_workspace_size(3, Hq, Hkv, d, tiers, 64)
+        assert got == up(n_slots * Hq * 4) + up(n_slots * Hq * d * 4)
+
+
 def test_decode_host_refusals(akv):
     """akv_decode_host checks its workspace, its flags and its host arrays before any launch;
     arrays that are not page-locked (here plain numpy memory) are AKV_ERR_NOT_PINNED."""
