@@ -287,23 +287,25 @@ akv_status akv_decode_host(const void* q_host, int B, int Hq, int Hkv, int d, fl
 
 /* ------------------------------------------------------------------------------------
  * akv_decode_static -- akv_decode without a workspace argument, for callers that cannot
- * allocate device memory when they decode (code inside a host function enqueued on a
- * stream, where CUDA forbids calls such as cudaMalloc; a plugin whose process memory pool
- * belongs to another framework; a serving loop that has frozen allocation so no call can
- * block on the allocator or synchronise the device).  The pages have no counterpart:
- * their engine always owns its memory.
+ * allocate device memory when they decode: a plugin whose process memory pool belongs to
+ * another framework, or a serving loop that has frozen allocation so that no call can block
+ * on the allocator or synchronise the device.  (It launches kernels, so like every CUDA
+ * call it must not be made from a host function enqueued on a stream.)  The pages have no
+ * counterpart: their engine always owns its memory.
  *
  * The scratch is a fixed array of AKV_DECODE_STATIC_MAX_BYTES in this library's device
- * memory, held by every GPU that loads the library until the process exits; the call
- * itself allocates no memory, on the device or the host (the first call that runs two tiers
- * side by side creates the internal stream and events akv_decode_attend describes).  A step
- * whose partials do not fit
- * (see akv_decode_workspace_size), or with more than AKV_DECODE_STATIC_MAX_SEQ sequences
- * or 8 tiers, returns AKV_ERR_BUDGET / AKV_ERR_UNSUPPORTED and launches nothing.  The
- * first call on each device looks up the array's device address while that device is
- * current, so make it before any stream capture.  Every call shares the array: it keeps
- * the last call's values, and calls whose work overlaps on the GPU race -- order them.
- * Arguments and results are those of akv_decode.
+ * memory, held by every GPU that loads the library until the process exits.  The first call
+ * on each device looks up the array's device address while that device is current; under
+ * CUDA's lazy module loading that lookup also loads the library's device code on the
+ * device, which reserves the array and may block.  So make one warm-up call on each device
+ * before freezing allocation or starting a stream capture.  After it, a call allocates no
+ * memory, on the device or the host (the first call that runs two tiers side by side also
+ * creates the internal stream and events akv_decode_attend describes).  A step whose
+ * partials do not fit (see akv_decode_workspace_size), or with more than
+ * AKV_DECODE_STATIC_MAX_SEQ sequences or 8 tiers, returns AKV_ERR_BUDGET /
+ * AKV_ERR_UNSUPPORTED and launches nothing.  Every call shares the array: it keeps the last
+ * call's values, and calls whose work overlaps on the GPU race -- order them.  Arguments and
+ * results are those of akv_decode, bit for bit.
  * ------------------------------------------------------------------------------------ */
 #define AKV_DECODE_STATIC_MAX_BYTES (8u << 20)
 #define AKV_DECODE_STATIC_MAX_SEQ 1024

@@ -13,11 +13,12 @@
 // consecutive items share their query).  Exact tier: NW = 8 chains per split, warp w runs
 // chain w of every item of the CTA back to back.  Compact tier: one chain per split, each
 // warp owns its own item range.  Every warp streams its steps through a private ring of
-// NST shared-memory stages that keeps prefetching across item boundaries.  Stages are filled by the copy engine, one lane issuing:
-// TMA tiles (cp.async.bulk.tensor, 128-byte swizzle) for BF16 rows, plain bulk copies
-// (cp.async.bulk) for compact code blocks; each stage completes on its own mbarrier.  Every
-// mbarrier wait is bounded: a wait that runs out sets AKV_EFLAG_TIMEOUT and the warp stops
-// computing, drains its copies (again bounded) and leaves.
+// NST shared-memory stages that keeps prefetching across item boundaries.  BF16 stages are
+// TMA tiles (cp.async.bulk.tensor, 128-byte swizzle) issued by one lane, each completing on
+// its own mbarrier; every mbarrier wait is bounded: a wait that runs out sets
+// AKV_EFLAG_TIMEOUT and the warp stops computing, drains its copies (again bounded) and
+// leaves.  Compact stages are the key and value blocks as stored, copied by all 32 lanes in
+// 16-byte cp.async.cg chunks, one commit group per step.
 //
 // Exact BF16 tier, per step (16 tokens):
 //   S^T (16 rows x 16 tokens) = q . K^T     A = q rows (heads), B = K rows via ldmatrix

@@ -1,21 +1,24 @@
 // akv_decode_static: the whole decode step for callers that cannot allocate device memory.
 //
-// akv_decode needs a scratch workspace for its split partials,
-// and leaves it to the caller to provide one.  Some callers have no way to get device
-// memory at the moment they decode: code running inside a host function enqueued on a
-// stream (where CUDA forbids API calls such as cudaMalloc), a plugin living in a process
-// whose memory pool belongs to another framework and is not shared with it, or a serving
-// loop that has frozen allocation so that no call can block on the allocator or
-// synchronise the device.  This entry point serves them: its scratch is a fixed array in
-// this library's device memory, so the call needs nothing beyond its inputs and outputs.
+// akv_decode needs a scratch workspace for its split partials, and leaves it to the caller
+// to provide one.  Some callers have no way to get device memory at the moment they decode:
+// a plugin living in a process whose memory pool belongs to another framework and is not
+// shared with it, or a serving loop that has frozen allocation so that no call can block on
+// the allocator or synchronise the device.  This entry point serves them: its scratch is a
+// fixed array in this library's device memory, so the call needs nothing beyond its inputs
+// and outputs.  (It is not for code running inside a host function enqueued on a stream:
+// CUDA forbids every runtime call there, and this one launches kernels.)
 //
 // The array is a file-scope __device__ object of AKV_DECODE_STATIC_MAX_BYTES.  Every GPU
 // that loads the library holds it until the process exits.  Host code cannot use the
 // array's name as a device address, so the first call on each device looks the address
 // up with cudaGetSymbolAddress while that device is current, and later calls on the
-// device reuse it; make that first call before any stream capture.  All calls share the
-// one array: it keeps whatever the last call left in it, and two calls whose work overlaps
-// on the GPU (two streams, say) race on the array -- order them.
+// device reuse it.  Under CUDA's lazy module loading that first lookup also loads this
+// library's device code on the device, which reserves the array and may block: make one
+// warm-up call before freezing allocation or starting a stream capture.  All calls share
+// the one array: it keeps whatever the last call left in it, and two calls whose work
+// overlaps on the GPU (two streams, say) race on the array -- order them.
+#include <cstdio>
 #include <mutex>
 
 #include "akv_internal.cuh"
@@ -24,16 +27,19 @@ namespace {
 
 __device__ __align__(256) uint8_t g_decode_scratch[AKV_DECODE_STATIC_MAX_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_decode_scratch, per device
+void* g_scratch_addr[akv::kMaxDevices];  // device address of g_decode_scratch, per device
 
 // The scratch's device address on the current device (looked up once per device).
 akv_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return akv::set_error(AKV_ERR_CUDA, cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return akv::set_error(AKV_ERR_UNSUPPORTED, "device index above 63");
+  if (dev < 0 || dev >= akv::kMaxDevices) {
+    char msg[96];
+    std::snprintf(msg, sizeof(msg), "akv_decode_static: device index %d is not below %d", dev, akv::kMaxDevices);
+    return akv::set_error(AKV_ERR_UNSUPPORTED, msg);
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
