@@ -191,3 +191,13 @@ def torch_student_t3_bf16(g, shape, device="cuda"):
     for _ in range(3):
         chi2.add_(torch.randn(shape, generator=g, device=device, dtype=torch.float32).square_())
     return (z / torch.sqrt(chi2 / 3.0)).to(torch.bfloat16).view(torch.int16)
+
+
+def torch_sequence_kv(wl: Workload, b: int, L: int, key_dist: str = "student_t", key: str = "kv", device="cuda"):
+    """K, V of sequence b, [Hkv, L, d] int16 tensors of BF16 bits, drawn on `device` from the
+    sequence's own seeded generator (keys Student-t(3) or N(0,1), values N(0,1)).  The same
+    call always returns the same bits, so a test can redraw any sequence of a full-size batch."""
+    g = torch_generator(wl.seed, wl.name, key, b, device=device)
+    shape = (wl.Hkv, L, wl.d)
+    k = torch_student_t3_bf16(g, shape, device) if key_dist == "student_t" else torch_normal_bf16(g, shape, device)
+    return k, torch_normal_bf16(g, shape, device)

@@ -236,10 +236,7 @@ class RaggedPaged:
         d, H = wl.d, wl.Hkv
         for b in range(self.B):
             L, c = int(lens[b]), int(cp_len[b])
-            g = synth.torch_generator(wl.seed, wl.name, "kv", b, device=device)
-            k = synth.torch_student_t3_bf16(g, (H, L, d), device) if self.key_dist == "student_t" \
-                else synth.torch_normal_bf16(g, (H, L, d), device)
-            v = synth.torch_normal_bf16(g, (H, L, d), device)
+            k, v = synth.torch_sequence_kv(wl, b, L, self.key_dist, device=device)
             if c > 0:
                 src = akv.Tier(akv.AKV_TIER_BF16, k, v, lens=[c], stride_seq=0, stride_head=L * d, stride_token=d)
                 dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True,
@@ -280,7 +277,7 @@ class StagedDecode:
 
     def __init__(self, wl: synth.Workload, device, layers: int | None = None, T: int | None = None,
                  chunk: int | None = None, max_steps: int = 8, n_buffers: int = 2, resident: bool = False,
-                 host_layers=None):
+                 host_layers=None, source: str = "host"):
         self.wl, self.device, self.resident = wl, device, resident
         self.L = wl.extra["layers"] if layers is None else layers
         self.T = wl.extra["T"] if T is None else T
@@ -291,12 +288,22 @@ class StagedDecode:
         cap = self.T + max_steps
         self.cap = -(-cap // self.chunk) * self.chunk
         if host_layers is None:
+            # source "host": numpy streams (the oracle can redraw any layer); "torch": seeded
+            # device generators, for full-size runs that need no oracle
             host_layers = []
             for layer in range(self.L):
-                k, v = synth.history_token_major(wl, layer, self.T)
                 h = torch.empty((self.cap, 2, H, d), dtype=torch.int16).pin_memory()
-                h[: self.T, 0] = torch.from_numpy(k.view(np.int16))
-                h[: self.T, 1] = torch.from_numpy(v.view(np.int16))
+                if source == "torch":
+                    g = synth.torch_generator(wl.seed, wl.name, "staged", layer, device=device)
+                    rows = torch.empty((self.T, 2, H, d), dtype=torch.int16, device=device)
+                    rows[:, 0] = synth.torch_normal_bf16(g, (self.T, H, d), device)
+                    rows[:, 1] = synth.torch_normal_bf16(g, (self.T, H, d), device)
+                    h[: self.T].copy_(rows)
+                    del rows
+                else:
+                    k, v = synth.history_token_major(wl, layer, self.T)
+                    h[: self.T, 0] = torch.from_numpy(k.view(np.int16))
+                    h[: self.T, 1] = torch.from_numpy(v.view(np.int16))
                 h[self.T:].zero_()  # rows the appended tokens will take (a reused pinned block holds old data)
                 host_layers.append(h)
         self.host = host_layers
