@@ -829,19 +829,20 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
     for i in range(n_warm):
         st.step(*inputs[i], variant, stream)
     torch.cuda.synchronize()
-    aged0, tok = st.aged_blocks, 0
-    st.encode_events = []
+    aged0 = st.aged_blocks
+    tok0 = int(st.c.sum() + st.win.sum())  # history tokens before the first timed step
     ctx.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(n_warm, n_steps):
-        tok += int(st.c.sum() + st.win.sum()) + wl.B
-        st.step(*inputs[i], variant, stream)
+        st.step(*inputs[i], variant, stream, sync_state=False)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = ctx.max(e0.elapsed_time(e1))
+    st._state()
     aged = st.aged_blocks - aged0
-    enc_us = [a.elapsed_time(b) * 1e3 for a, b in st.encode_events]
+    # step j attends every earlier token plus the B it appends
+    tok = sum(tok0 + wl.B * (j + 1) for j in range(steps))
     value = tok * ctx.world / (ms * 1e-3)
     err = int(st.err.item())
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ctx.world, "steps": steps,
@@ -851,10 +852,10 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
                                    "32768 tokens, newest 2048-2063 BF16 in 16-token ring pages, the rest 4-bit "
                                    "code pages; one token appended per step, full window pages encoded into "
                                    "the compact tier", "parallelism": f"independent replicas x{ctx.world}",
-                       "variant": args.variant, "timing": "CUDA events around whole steps"},
-            "aged_blocks_in_timed_steps": int(aged) * wl.Hkv, "aging_events": len(enc_us),
-            "aging_encode_us_avg": sum(enc_us) / max(1, len(enc_us)),
-            "e2e": None, "gpu_launches": steps * 3 + int(aged > 0) * (aged // wl.B),
+                       "variant": args.variant, "timing": "CUDA events around whole steps",
+                       "step": "one akv_aging_step call (append, aging encode, attention launches, merge)"},
+            "aged_pages_in_timed_steps": int(aged),
+            "e2e": None, "gpu_launches": steps * 4 + 2 * int(aged > 0) * (aged // wl.B),
             "device_error_word": err}
 
 

@@ -363,7 +363,9 @@ akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, i
  *
  * akv_stage_chunk: take the next buffer; make sure every event on its list has fired;
  *   copy `bytes` from pinned_src (page-locked host memory, else AKV_ERR_NOT_PINNED) with
- *   cudaMemcpyAsync on copy_stream; record the copy's event.  bytes larger than one
+ *   cudaMemcpyAsync on copy_stream, ordered after every akv_stage_writeback of this stager
+ *   still in flight whose host range overlaps the source (copy_stream waits for it on the
+ *   device); record the copy's event.  bytes larger than one
  *   buffer gives AKV_ERR_BUDGET; bytes == 0 acquires the buffer without copying (the
  *   caller fills it on the device).  timeout_ms >= 0: the host polls the events for at most
  *   timeout_ms and returns AKV_ERR_TIMEOUT, leaving the buffer untouched, if one is still
@@ -387,6 +389,99 @@ akv_status akv_stager_release(akv_stager* st, int buf_index, akv_stream_t consum
 akv_status akv_stage_writeback(akv_stager* st, int buf_index, size_t offset, void* pinned_dst, size_t bytes,
                                akv_stream_t stream);
 akv_status akv_stager_destroy(akv_stager* st);
+
+/* ------------------------------------------------------------------------------------
+ * akv_staged_decode -- one decode step of one layer whose history lives in pinned host
+ * memory, in one call ("Context beyond VRAM", "What I built": the fence-safe staging
+ * pipeline -- the step appends the new K/V, stages the history through the bounded device
+ * region, attends and merges, and a buffer is reused only after everything that touched it
+ * has finished).
+ *
+ * hist->host holds the layer's rows from token 0, pinned:
+ *   AKV_TIER_BF16:   token rows [n][K | V][Hkv][d] bf16 (2 Hkv d 2 bytes per token);
+ *   AKV_TIER_CODES4: 16-token block rows [n / 16][K | V][Hkv][AKV_CODES4_BLOCK_BYTES(d)].
+ * The history is cut into chunks of hist->chunk_tokens tokens (a multiple of split_tokens,
+ * and for CODES4 of 16); chunk c is staged with akv_stage_chunk on copy_stream, attended on
+ * compute_stream into slots [c chunk / split, ...) and released.  new_row (device bf16
+ * [2][Hkv][d], BF16 histories only, may be NULL) is the new token: it is appended at
+ * position hist->n_tokens -- written into its staged chunk before that chunk is attended --
+ * and written back to its host row (so the next step's copy of that chunk waits for it).
+ * window (may be NULL): a device BF16 tier of one sequence attended after the history into
+ * the following slots (the exact window of a staged hybrid history; the caller appends
+ * to it).  The splits of the history, then of the window, are merged in order into o, lse
+ * (device float32 [Hq][d], [Hq]).  o_part / lse_part: device scratch of n_slots slots.
+ * Results equal akv_decode_attend + akv_merge_lse over the same tokens and split layout, bit
+ * for bit (a staged run equals a resident run).  Refusals: as the calls it makes, plus
+ * AKV_ERR_BUDGET when n_slots is too small; an error part-way leaves earlier chunks enqueued.
+ * ------------------------------------------------------------------------------------ */
+typedef struct akv_staged_history {
+  int32_t kind;                 /* AKV_TIER_BF16 or AKV_TIER_CODES4 */
+  int32_t chunk_tokens;         /* tokens per staged chunk */
+  const void* host;             /* pinned host rows from token 0 */
+  int64_t n_tokens;             /* tokens in the history before this step's append */
+  uint32_t rotation_signs[4];   /* CODES4: the rotation signs the codes were written with */
+} akv_staged_history;
+
+akv_status akv_staged_decode(akv_stager* stager, const akv_staged_history* hist, const void* q, int Hq, int Hkv,
+                             int d, float softmax_scale, int split_tokens, const void* new_row,
+                             const akv_tier* window, float* o_part, float* lse_part, int64_t n_slots, float* o,
+                             float* lse, int variant, int32_t* err_word, akv_stream_t copy_stream,
+                             akv_stream_t compute_stream);
+
+/* ------------------------------------------------------------------------------------
+ * Window aging -- a live hybrid batch whose exact window ages into the compact tier during
+ * decode ("Context beyond VRAM", "What I built": recent context exact, older history in
+ * the compact form), one call per step.
+ *
+ * Sequence b keeps compact_len[b] compact tokens (a multiple of 16) and window_len[b] in
+ * [W, W + 16) exact tokens, W = window_tokens.  The window is a ring of ring_pages
+ * (>= W / 16 + 2) pages of 16 BF16 tokens: window pool page b * ring_pages + (head + j) %
+ * ring_pages holds the window's logical page j, where head = ring_head[b] is the ring slot
+ * of its first page, and the window tier's page-table row b (ring_pages entries, device)
+ * must say so.  The compact tier's page-table row b holds page_lists[b][0 ..
+ * compact_len[b] / 16); as the sequence ages it takes page_lists[b][compact_len[b] / 16],
+ * then the next.
+ *
+ * akv_aging_step, for every sequence: appends the new token (k_new, v_new: device bf16
+ * [B][Hkv][d]) at window position window_len[b]; a window that reaches W + 16 tokens
+ * encodes its oldest page into the sequence's next code page (akv_encode_history), enters
+ * that page in the compact page table and rotates its window page-table row (both written
+ * on the device by the call) -- then attends both tiers with the standard slot layout
+ * (akv_plan_slots) into o_part / lse_part (n_slots slots) and merges into o, lse (device
+ * float32 [B][Hq][d], [B][Hq]).  Everything is enqueued on `stream`; the context keeps the
+ * lengths on the host.  lists_dev: device int32 scratch of 2 B entries (the encode's page
+ * lists).  A sequence with no code page left is refused (AKV_ERR_BUDGET) before anything is
+ * enqueued.  The tiers' lens and slot_base are ignored.  Results equal the same calls made
+ * one by one.  akv_aging_state reads the current lengths, ring heads and the number of pages
+ * aged so far (host arrays of B entries, each may be NULL).  The context holds copies of
+ * every host array of the description; it owns no device memory.
+ * ------------------------------------------------------------------------------------ */
+typedef struct akv_aging akv_aging;
+
+typedef struct akv_aging_desc {
+  int32_t B, Hq, Hkv, d, split_tokens;
+  float softmax_scale;
+  int32_t window_tokens;             /* W: a positive multiple of 16 */
+  int32_t ring_pages;                /* window pages per sequence */
+  akv_tier window;                   /* BF16, paged: B * ring_pages pool pages; page_table device [B][ring_pages] */
+  akv_tier compact;                  /* CODES4, paged; page_table device [B][page_table_stride] */
+  const int32_t* compact_len;        /* host [B] */
+  const int32_t* window_len;         /* host [B] */
+  const int32_t* ring_head;          /* host [B] */
+  const int32_t* const* page_lists;  /* host [B] arrays of code pages, in the order they are taken */
+  const int32_t* page_list_len;      /* host [B] */
+  int32_t* lists_dev;                /* device int32 [2 B] scratch */
+  float* o_part;                     /* device [n_slots][Hq][d] */
+  float* lse_part;                   /* device [n_slots][Hq] */
+  int64_t n_slots;
+} akv_aging_desc;
+
+akv_status akv_aging_create(const akv_aging_desc* desc, akv_aging** out);
+akv_status akv_aging_step(akv_aging* ctx, const void* q, const void* k_new, const void* v_new, float* o, float* lse,
+                          int variant, int32_t* err_word, akv_stream_t stream);
+akv_status akv_aging_state(const akv_aging* ctx, int32_t* compact_len, int32_t* window_len, int32_t* ring_head,
+                           int64_t* aged_pages);
+akv_status akv_aging_destroy(akv_aging* ctx);
 
 #ifdef __cplusplus
 }

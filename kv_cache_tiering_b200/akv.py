@@ -82,6 +82,37 @@ class AkvTierC(ctypes.Structure):
     ]
 
 
+class AkvStagedHistoryC(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("chunk_tokens", ctypes.c_int32),
+        ("host", _p),
+        ("n_tokens", ctypes.c_int64),
+        ("rotation_signs", ctypes.c_uint32 * 4),
+    ]
+
+
+class AkvAgingDescC(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("split_tokens", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("window_tokens", ctypes.c_int32),
+        ("ring_pages", ctypes.c_int32),
+        ("window", AkvTierC),
+        ("compact", AkvTierC),
+        ("compact_len", _p),
+        ("window_len", _p),
+        ("ring_head", _p),
+        ("page_lists", ctypes.POINTER(_p)),
+        ("page_list_len", _p),
+        ("lists_dev", _p),
+        ("o_part", _p),
+        ("lse_part", _p),
+        ("n_slots", ctypes.c_int64),
+    ]
+
+
 def _sig(name, res, *args):
     f = getattr(lib, name)
     f.restype = res
@@ -128,12 +159,20 @@ _sig("akv_stager_use", ctypes.c_int, _p, ctypes.c_int, _p)
 _sig("akv_stager_release", ctypes.c_int, _p, ctypes.c_int, _p)
 _sig("akv_stage_writeback", ctypes.c_int, _p, ctypes.c_int, ctypes.c_size_t, _p, ctypes.c_size_t, _p)
 _sig("akv_stager_destroy", ctypes.c_int, _p)
+_sig("akv_staged_decode", ctypes.c_int, _p, ctypes.POINTER(AkvStagedHistoryC), _p, ctypes.c_int, ctypes.c_int,
+     ctypes.c_int, ctypes.c_float, ctypes.c_int, _p, ctypes.POINTER(AkvTierC), _p, _p, ctypes.c_int64, _p, _p,
+     ctypes.c_int, _p, _p, _p)
+_sig("akv_aging_create", ctypes.c_int, ctypes.POINTER(AkvAgingDescC), ctypes.POINTER(_p))
+_sig("akv_aging_step", ctypes.c_int, _p, _p, _p, _p, _p, _p, ctypes.c_int, _p, _p)
+_sig("akv_aging_state", ctypes.c_int, _p, _p, _p, _p, ctypes.POINTER(ctypes.c_int64))
+_sig("akv_aging_destroy", ctypes.c_int, _p)
 
 EXPORTED = [
     "akv_abi_version", "akv_last_error", "akv_status_string", "akv_error_word_status", "akv_centroids_f16",
     "akv_plan_slots", "akv_encode_history", "akv_decode_attend", "akv_merge_lse", "akv_decode_workspace_size",
     "akv_decode", "akv_decode_host_workspace_size", "akv_decode_host", "akv_stager_create",
     "akv_stage_chunk", "akv_stager_use", "akv_stager_release", "akv_stage_writeback", "akv_stager_destroy",
+    "akv_staged_decode", "akv_aging_create", "akv_aging_step", "akv_aging_state", "akv_aging_destroy",
 ]
 
 
@@ -381,6 +420,69 @@ class Stager:
         if self._h:
             h, self._h = self._h, None
             _check(lib.akv_stager_destroy(h))
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def _signs_c(bits: int):
+    return (ctypes.c_uint32 * 4)(*[(int(bits) >> (32 * i)) & 0xFFFFFFFF for i in range(4)])
+
+
+def akv_staged_decode(stager: "Stager", kind: int, host, n_tokens: int, chunk_tokens: int, q, Hq: int, Hkv: int,
+                      d: int, softmax_scale: float, split_tokens: int, new_row, window, o_part, lse_part,
+                      n_slots: int, o, lse, variant: int = AKV_VARIANT_AUTO, err_word=None, copy_stream=None,
+                      compute_stream=None, rotation_signs: int = 0) -> None:
+    """One staged decode step of one layer (see akv_staged_decode in include/akv.h)."""
+    h = AkvStagedHistoryC(kind, chunk_tokens, _ptr(host), n_tokens, _signs_c(rotation_signs))
+    w = None
+    if window is not None:
+        wa = _tier_array([window])
+        w = wa.arr
+    _check(lib.akv_staged_decode(stager._h, ctypes.byref(h), _ptr(q), Hq, Hkv, d, float(softmax_scale), split_tokens,
+                                 _ptr(new_row), w, _ptr(o_part), _ptr(lse_part), int(n_slots), _ptr(o), _ptr(lse),
+                                 variant, _ptr(err_word), _stream(copy_stream), _stream(compute_stream)))
+
+
+class Aging:
+    """Owner of an ``akv_aging`` context (see include/akv.h): a live hybrid batch whose exact
+    window ages into the compact tier, one akv_aging_step call per decode step."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, d: int, split_tokens: int, softmax_scale: float,
+                 window_tokens: int, ring_pages: int, window: Tier, compact: Tier, compact_len, window_len,
+                 ring_head, page_lists, lists_dev, o_part, lse_part, n_slots: int):
+        lists = [_host_i32(x) for x in page_lists]
+        lens = [_host_i32(x) for x in (compact_len, window_len, ring_head)]
+        list_len = _host_i32([len(x) for x in lists])
+        ptrs = (_p * max(1, B))(*[x.ctypes.data for x in lists])
+        wc, cc = window.c(), compact.c()
+        self._keep = [lists, lens, list_len, ptrs, window._keep, compact._keep]
+        desc = AkvAgingDescC(B, Hq, Hkv, d, split_tokens, float(softmax_scale), window_tokens, ring_pages, wc, cc,
+                             lens[0].ctypes.data, lens[1].ctypes.data, lens[2].ctypes.data, ptrs,
+                             list_len.ctypes.data, _ptr(lists_dev), _ptr(o_part), _ptr(lse_part), int(n_slots))
+        h = _p()
+        _check(lib.akv_aging_create(ctypes.byref(desc), ctypes.byref(h)))
+        self._h = h
+        self.B = B
+
+    def step(self, q, k_new, v_new, o, lse, variant: int = AKV_VARIANT_AUTO, err_word=None, stream=None) -> None:
+        _check(lib.akv_aging_step(self._h, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(o), _ptr(lse), variant,
+                                  _ptr(err_word), _stream(stream)))
+
+    def state(self):
+        """(compact lengths, window lengths, ring heads, pages aged so far)."""
+        c, w, r = (np.zeros(self.B, np.int32) for _ in range(3))
+        aged = ctypes.c_int64(0)
+        _check(lib.akv_aging_state(self._h, c.ctypes.data, w.ctypes.data, r.ctypes.data, ctypes.byref(aged)))
+        return c, w, r, aged.value
+
+    def destroy(self) -> None:
+        if self._h:
+            h, self._h = self._h, None
+            _check(lib.akv_aging_destroy(h))
 
     def __del__(self):
         try:

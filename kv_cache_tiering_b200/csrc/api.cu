@@ -812,11 +812,19 @@ struct akv_stager {
     std::vector<cudaEvent_t> pending;  // copies and consumers since the last fill
     cudaEvent_t ready = nullptr;       // the latest fill's copy
   };
+  // A write-back into host memory that may still be in flight: a later chunk whose source
+  // overlaps [lo, hi) must be copied after it.
+  struct HostWrite {
+    const uint8_t* lo;
+    const uint8_t* hi;
+    cudaEvent_t done;
+  };
   uint8_t* region = nullptr;
   size_t buf_bytes = 0;
   int n = 0;
   int next = 0;
   std::vector<Buffer> bufs;
+  std::vector<HostWrite> host_writes;
   std::vector<cudaEvent_t> free_events;
   std::vector<cudaEvent_t> all_events;
 };
@@ -895,6 +903,25 @@ akv_status akv_stage_chunk(akv_stager* st, const void* pinned_src, size_t bytes,
     cudaError_t e = cudaStreamWaitEvent(cs, ev, 0);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   }
+  // the copy reads host bytes that an earlier write-back may still be writing: order it
+  // after every such write-back; write-backs that have completed are forgotten
+  const uint8_t* src_lo = static_cast<const uint8_t*>(pinned_src);
+  for (size_t i = 0; i < st->host_writes.size();) {
+    akv_stager::HostWrite& w = st->host_writes[i];
+    const cudaError_t q = cudaEventQuery(w.done);
+    if (q == cudaSuccess) {
+      st->free_events.push_back(w.done);
+      w = st->host_writes.back();
+      st->host_writes.pop_back();
+      continue;
+    }
+    if (q != cudaErrorNotReady) return cuda_fail(q, "cudaEventQuery");
+    if (bytes && w.lo < src_lo + bytes && src_lo < w.hi) {
+      const cudaError_t e = cudaStreamWaitEvent(cs, w.done, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    }
+    ++i;
+  }
   // a wait binds to the event's latest record at the time of the call, so the events
   // can be recycled now
   for (cudaEvent_t ev : buf.pending) st->free_events.push_back(ev);
@@ -952,6 +979,14 @@ akv_status akv_stage_writeback(akv_stager* st, int buf_index, size_t offset, voi
   const uint8_t* src = st->region + (size_t)buf_index * st->buf_bytes + offset;
   if ((e = cudaMemcpyAsync(pinned_dst, src, bytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
     return cuda_fail(e, "cudaMemcpyAsync D2H");
+  cudaEvent_t done;
+  if ((e = take_event(st, &done)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  if ((e = cudaEventRecord(done, s)) != cudaSuccess) {
+    st->free_events.push_back(done);
+    return cuda_fail(e, "cudaEventRecord");
+  }
+  const uint8_t* lo = static_cast<const uint8_t*>(pinned_dst);
+  st->host_writes.push_back({lo, lo + bytes, done});
   return akv_stager_release(st, buf_index, stream);
 }
 
@@ -963,6 +998,10 @@ akv_status akv_stager_destroy(akv_stager* st) {
       cudaError_t e = cudaEventSynchronize(ev);
       if (e != cudaSuccess && result == AKV_OK) result = cuda_fail(e, "cudaEventSynchronize");
     }
+  for (auto& w : st->host_writes) {
+    cudaError_t e = cudaEventSynchronize(w.done);
+    if (e != cudaSuccess && result == AKV_OK) result = cuda_fail(e, "cudaEventSynchronize");
+  }
   for (cudaEvent_t ev : st->all_events) cudaEventDestroy(ev);
   delete st;
   return result == AKV_OK ? ok() : result;

@@ -322,7 +322,6 @@ class StagedDecode:
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
         self.steps_done = 0
         self.h2d_bytes = 0
-        self._wb_events = [None] * self.L  # per layer: the last write-back of an appended row
 
     def inputs(self, step: int):
         """Device q [L][Hq][d] and new rows [L][2][Hkv][d] of decode step ``step``."""
@@ -331,7 +330,12 @@ class StagedDecode:
         return to_dev_bits(q, self.device), to_dev_bits(new, self.device)
 
     def step(self, q, new_rows, variant=akv.AKV_VARIANT_AUTO, timeout_ms: int = -1):
-        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device)."""
+        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device).
+        Staged: one akv_staged_decode call per layer.  Resident: the same attention calls over
+        the same chunks in device memory (the bit-identity comparison run)."""
+        if not self.resident:
+            self._step_staged(q, new_rows, variant)
+            return
         wl, H, d = self.wl, self.wl.Hkv, self.wl.d
         pos = self.T + self.steps_done          # position of the appended token
         n_tok = pos + 1
@@ -340,29 +344,15 @@ class StagedDecode:
         n_split = -(-n_tok // wl.split_tokens)
         per_chunk = self.chunk // wl.split_tokens
         rb = self.row_bytes
-        # the step's inputs come from the caller's stream
-        cs.wait_stream(torch.cuda.current_stream(self.device))
+        cs.wait_stream(torch.cuda.current_stream(self.device))  # the step's inputs
         for layer in range(self.L):
             new_row = new_rows[layer].reshape(-1).view(torch.uint8)
+            store = self.dev_layers[layer].view(torch.uint8).reshape(-1)
             for c in range(n_chunks):
                 tok0 = c * self.chunk
                 ntc = min(self.chunk, n_tok - tok0)
-                have = min(self.chunk, pos - tok0)  # rows already in the host copy
                 appends = tok0 <= pos < tok0 + self.chunk
-                buf = None
-                if self.resident:
-                    store = self.dev_layers[layer].view(torch.uint8).reshape(-1)
-                    off = tok0 * rb
-                else:
-                    src = self.host[layer].data_ptr() + tok0 * rb
-                    if tok0 <= pos - 1 < tok0 + self.chunk and self._wb_events[layer] is not None:
-                        # the previous step wrote row pos - 1 back to this chunk's host span
-                        self.copy_stream.wait_event(self._wb_events[layer])
-                    buf, dev = self.stager.stage_chunk(src, have * rb, self.copy_stream, timeout_ms)
-                    self.h2d_bytes += have * rb
-                    self.stager.use(buf, cs)
-                    store = self.region
-                    off = dev - self.region.data_ptr()
+                off = tok0 * rb
                 base = store.data_ptr() + off
                 with torch.cuda.stream(cs):
                     if appends:  # the new token's row goes into the chunk that holds its position
@@ -371,20 +361,25 @@ class StagedDecode:
                                     slot_base=[c * per_chunk], stride_seq=0, stride_head=d, stride_token=2 * H * d)
                     akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
                                           self.lse_part, self.o_part.shape[0], variant, self.err, cs)
-                    if appends:  # write the new row back to the authoritative host copy
-                        if self.resident:
-                            self.host[layer][pos].view(torch.uint8).reshape(-1).copy_(
-                                store[off + (pos - tok0) * rb: off + (pos - tok0 + 1) * rb], non_blocking=True)
-                        else:
-                            self.stager.writeback(buf, (pos - tok0) * rb, self.host[layer].data_ptr() + pos * rb,
-                                                  rb, cs)
-                            ev = torch.cuda.Event()
-                            ev.record(cs)
-                            self._wb_events[layer] = ev
-                if buf is not None:
-                    self.stager.release(buf, cs)
+                    if appends:  # write the new row back to the host copy
+                        self.host[layer][pos].view(torch.uint8).reshape(-1).copy_(
+                            store[off + (pos - tok0) * rb: off + (pos - tok0 + 1) * rb], non_blocking=True)
             akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [n_split], 1, wl.Hq, d,
                               self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
+        torch.cuda.current_stream(self.device).wait_stream(cs)  # the results, for the caller's stream
+        self.steps_done += 1
+
+    def _step_staged(self, q, new_rows, variant):
+        wl, H, d = self.wl, self.wl.Hkv, self.wl.d
+        pos = self.T + self.steps_done
+        cs = self.compute_stream
+        cs.wait_stream(torch.cuda.current_stream(self.device))  # the step's inputs
+        for layer in range(self.L):
+            akv.akv_staged_decode(self.stager, akv.AKV_TIER_BF16, self.host[layer], pos, self.chunk, q[layer], wl.Hq,
+                                  H, d, wl.scale, wl.split_tokens, new_rows[layer], None, self.o_part, self.lse_part,
+                                  self.o_part.shape[0], self.o[layer:layer + 1], self.lse[layer:layer + 1], variant,
+                                  self.err, self.copy_stream, cs)
+            self.h2d_bytes += pos * self.row_bytes
         torch.cuda.current_stream(self.device).wait_stream(cs)  # the results, for the caller's stream
         self.steps_done += 1
 
@@ -495,7 +490,10 @@ class StagedHybridDecode:
         return to_dev_bits(q, self.device), to_dev_bits(new, self.device)
 
     def step(self, q, new_rows, variant=akv.AKV_VARIANT_AUTO, timeout_ms: int = -1):
-        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device)."""
+        """One decode step over all layers; q [L][Hq][d], new_rows [L][2][Hkv][d] (device).
+        Staged: the new row joins the device window, then one akv_staged_decode call per layer
+        stages and attends the compact history, attends the window and merges.  Resident: the
+        same attention calls over the compact rows in device memory (the comparison run)."""
         wl, H, d = self.wl, self.wl.Hkv, self.wl.d
         cs = self.compute_stream
         nw = self.W + self.steps_done + 1           # window tokens including the appended one
@@ -507,28 +505,25 @@ class StagedHybridDecode:
             win = self.win[layer]
             with torch.cuda.stream(cs):
                 win[nw - 1].copy_(new_rows[layer])
+            wb = win.data_ptr()
+            wtier = akv.Tier(akv.AKV_TIER_BF16, wb, wb + H * d * 2, lens=[nw], slot_base=[self.n_cslots],
+                             stride_seq=0, stride_head=d, stride_token=2 * H * d)
+            if not self.resident:
+                akv.akv_staged_decode(self.stager, akv.AKV_TIER_CODES4, self.host[layer], self.Tc, self.chunk,
+                                      q[layer], wl.Hq, H, d, wl.scale, wl.split_tokens, None, wtier, self.o_part,
+                                      self.lse_part, self.o_part.shape[0], self.o[layer:layer + 1],
+                                      self.lse[layer:layer + 1], variant, self.err, self.copy_stream, cs)
+                self.h2d_bytes += self.nrows * self.crow
+                continue
             for c in range(n_chunks):
                 tok0 = c * self.chunk
                 ntc = min(self.chunk, self.Tc - tok0)
-                row0, nrow = tok0 // 16, -(-ntc // 16)
-                buf = None
-                if self.resident:
-                    base = self.host[layer].data_ptr() + row0 * self.crow
-                else:
-                    buf, base = self.stager.stage_chunk(self.host[layer].data_ptr() + row0 * self.crow,
-                                                        nrow * self.crow, self.copy_stream, timeout_ms)
-                    self.h2d_bytes += nrow * self.crow
-                    self.stager.use(buf, cs)
+                base = self.host[layer].data_ptr() + (tok0 // 16) * self.crow
                 tier = akv.Tier(akv.AKV_TIER_CODES4, base, base + H * self.bb, lens=[ntc], slot_base=[c * per_chunk],
                                 stride_seq=0, stride_head=1, stride_token=2 * H)
                 akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
                                       self.lse_part, self.o_part.shape[0], variant, self.err, cs)
-                if buf is not None:
-                    self.stager.release(buf, cs)
-            wb = win.data_ptr()
-            tier = akv.Tier(akv.AKV_TIER_BF16, wb, wb + H * d * 2, lens=[nw], slot_base=[self.n_cslots],
-                            stride_seq=0, stride_head=d, stride_token=2 * H * d)
-            akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [tier], wl.split_tokens, self.o_part,
+            akv.akv_decode_attend(q[layer], 1, wl.Hq, H, d, wl.scale, [wtier], wl.split_tokens, self.o_part,
                                   self.lse_part, self.o_part.shape[0], variant, self.err, cs)
             akv.akv_merge_lse(self.o_part, self.lse_part, self.o_part.shape[0], [0], [self.n_cslots + n_wsplit], 1,
                               wl.Hq, d, self.o[layer:layer + 1], self.lse[layer:layer + 1], cs)
@@ -615,32 +610,27 @@ class AgingHybrid:
         self.o = torch.empty((self.B, wl.Hq, d), dtype=torch.float32, device=device)
         self.lse = torch.empty((self.B, wl.Hq), dtype=torch.float32, device=device)
         self.q = to_dev_bits(synth.queries(wl, B=self.B), device)
-        self._cp_host = torch.empty(self.cp_table_np.shape, dtype=torch.int32).pin_memory()
-        self._ex_host = torch.empty(self.ex_table_np.shape, dtype=torch.int32).pin_memory()
-        self._enc_host = torch.empty((self.B, 2), dtype=torch.int32).pin_memory()
         self._enc_dev = torch.empty((self.B, 2), dtype=torch.int32, device=device)
-        self._tables_done = torch.cuda.Event()
-        self._tables_done.record(torch.cuda.current_stream(device))
         self.steps_done = 0
+        # the step runs in the library: one akv_aging_step call appends, ages full window
+        # pages into the compact tier, attends both tiers and merges
+        self.ctx = akv.Aging(self.B, wl.Hq, H, d, wl.split_tokens, wl.scale, W, self.R, self._exact_tier(),
+                             akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=self.c.astype(np.int32),
+                                      paged=True, page_table=self.cp_table,
+                                      page_table_stride=self.cp_table_np.shape[1], n_pages=self.n_cp,
+                                      stride_seq=H, stride_head=1),
+                             self.c.astype(np.int32), self.win.astype(np.int32), self.ring0.astype(np.int32),
+                             self.owned, self._enc_dev, self.o_part, self.lse_part, self.o_part.shape[0])
+        self._aged0 = int(self.c.sum() // 16)
         self.aged_blocks = 0
-        self.encode_events = None  # a list: every aging encode is bracketed by timing events
-        # host arrays the marshalled tiers point to, updated in place every step: lengths, the
-        # append positions and the slot plan (replanned only when a tier's split count changes)
-        H = wl.Hkv
-        self._cp_len = np.zeros(self.B, np.int32)
-        self._ex_len = np.zeros(self.B, np.int32)
-        self._pos = np.zeros(self.B, np.int32)
-        self._cp_base = np.zeros(self.B, np.int32)
-        self._ex_base = np.zeros(self.B, np.int32)
-        self._seq_base = np.zeros(self.B, np.int32)
-        self._seq_n = np.zeros(self.B, np.int32)
-        self._n_slots = 0
-        self._plan_counts = None
-        codes = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=self._cp_len, slot_base=self._cp_base,
-                         paged=True, page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1],
-                         n_pages=self.n_cp, stride_seq=H, stride_head=1)
-        self._attend_tiers = akv.TierArray([codes, self._exact_tier(self._ex_len, self._ex_base)])
-        self._append_tier = akv.TierArray([self._exact_tier(self._ex_len)])
+
+    def _state(self):
+        c, w, r, _ = self.ctx.state()
+        self.c, self.win, self.ring0 = c.astype(np.int64), w.astype(np.int64), r.astype(np.int64)
+        n_pages = self.c // 16
+        for b in range(self.B):
+            self.cp_table_np[b, :n_pages[b]] = self.owned[b][:n_pages[b]]
+        self.aged_blocks = int(n_pages.sum()) - self._aged0
 
     def inputs(self, step: int):
         """Device q [B][Hq][d] and new K, V rows [B][Hkv][d] of decode step ``step``."""
@@ -656,68 +646,10 @@ class AgingHybrid:
                         slot_base=slot_base, paged=True, page_table=self.ex_table, page_table_stride=self.R,
                         n_pages=self.B * self.R, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
 
-    def _ex_row(self, b: int) -> np.ndarray:
-        return np.array([b * self.R + (self.ring0[b] + j) % self.R for j in range(self.R)], np.int32)
-
-    def step(self, q, k_new, v_new, variant=akv.AKV_VARIANT_AUTO, stream=None):
-        """Append one token per sequence, age full window pages, attend both tiers, merge."""
-        wl, H, d, B = self.wl, self.wl.Hkv, self.wl.d, self.B
-        dev = self.device
-        # 1. append: token win[b] of the window, through the window's page table
-        self._ex_len[:] = self.win
-        self._pos[:] = self.win
-        akv.akv_append_tokens(self._append_tier, self._pos, B, H, d, k_new, v_new, self.err, stream)
-        self.win += 1
-        # 2. age: a window of W + 16 tokens hands its oldest page to the compact tier
-        aging = [b for b in range(B) if self.win[b] >= self.W + 16]
-        if aging:
-            n = len(aging)
-            self._tables_done.synchronize()   # the pinned buffers' previous uploads have finished
-            enc = self._enc_host[:n]
-            for i, b in enumerate(aging):
-                enc[i, 0] = b * self.R + self.ring0[b]                  # oldest window page
-                enc[i, 1] = int(self.owned[b][self.c[b] // 16])         # the next code page
-                self.cp_table_np[b, int(self.c[b] // 16)] = enc[i, 1]
-                self.c[b] += 16
-                self.ring0[b] = (self.ring0[b] + 1) % self.R
-                self.win[b] -= 16
-                self.ex_table_np[b] = self._ex_row(b)
-            self._cp_host.copy_(torch.from_numpy(self.cp_table_np))
-            self._ex_host.copy_(torch.from_numpy(self.ex_table_np))
-            cur = torch.cuda.current_stream(dev) if stream is None else stream
-            with torch.cuda.stream(cur):
-                self._enc_dev[:n].copy_(enc, non_blocking=True)
-                ptr = self._enc_dev.data_ptr()
-                # column 0 of the page lists addresses the source pages, column 1 the destination
-                src = akv.Tier(akv.AKV_TIER_BF16, self.ex_k, self.ex_v, lens=[16] * n, paged=True, page_table=ptr,
-                               page_table_stride=2, n_pages=B * self.R, stride_seq=H * 16 * d, stride_head=16 * d,
-                               stride_token=d)
-                dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[16] * n, paged=True,
-                               page_table=ptr + 4, page_table_stride=2, n_pages=self.n_cp, stride_seq=H,
-                               stride_head=1)
-                if self.encode_events is not None:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(cur)
-                akv.akv_encode_history(src, dst, n, H, d, self.err, cur)
-                if self.encode_events is not None:
-                    e1.record(cur)
-                    self.encode_events.append((e0, e1))
-                self.cp_table.copy_(self._cp_host, non_blocking=True)
-                self.ex_table.copy_(self._ex_host, non_blocking=True)
-                self._tables_done.record(cur)
-            self.aged_blocks += n
-        # 3. attend both tiers into their planned slots, then merge
-        self._cp_len[:] = self.c
-        self._ex_len[:] = self.win
-        split = wl.split_tokens
-        counts = ((self._cp_len + split - 1) // split, (self._ex_len + split - 1) // split)
-        if self._plan_counts is None or any(not np.array_equal(a, b) for a, b in zip(counts, self._plan_counts)):
-            bases, seq_base, seq_n, self._n_slots = akv.plan_slots([self._cp_len, self._ex_len], split)
-            self._cp_base[:], self._ex_base[:] = bases[0], bases[1]
-            self._seq_base[:], self._seq_n[:] = seq_base, seq_n
-            self._plan_counts = counts
-        akv.akv_decode_attend(q, B, wl.Hq, H, d, wl.scale, self._attend_tiers, split, self.o_part, self.lse_part,
-                              self._n_slots, variant, self.err, stream)
-        akv.akv_merge_lse(self.o_part, self.lse_part, self._n_slots, self._seq_base, self._seq_n, B, wl.Hq, d, self.o,
-                          self.lse, stream)
+    def step(self, q, k_new, v_new, variant=akv.AKV_VARIANT_AUTO, stream=None, sync_state: bool = True):
+        """Append one token per sequence, age full window pages, attend both tiers, merge:
+        one akv_aging_step call.  sync_state=False skips reading the lengths back."""
+        self.ctx.step(q, k_new, v_new, self.o, self.lse, variant, self.err, stream)
         self.steps_done += 1
+        if sync_state:
+            self._state()

@@ -228,3 +228,64 @@ def test_header_is_plain_c():
     r = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-x", "c", "-",
                         "-I", os.path.join(root, "include")], input=src, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_staged_decode_refusals(akv):
+    """akv_staged_decode validates before it stages or launches anything."""
+    st = akv.Stager(0x100000, 1 << 20, 2)  # host bookkeeping only
+    host = np.zeros(4096, dtype=np.uint8)
+    common = dict(q=0x1000, Hq=32, Hkv=8, d=128, softmax_scale=0.1, split_tokens=512, o_part=0x2000,
+                  lse_part=0x3000, n_slots=64, o=0x4000, lse=0x5000)
+
+    def call(**kw):
+        args = dict(common, kind=akv.AKV_TIER_BF16, host=host, n_tokens=100, chunk_tokens=4096, new_row=None,
+                    window=None)
+        args.update(kw)
+        with pytest.raises(akv.AkvError) as e:
+            akv.akv_staged_decode(st, **args)
+        return e.value.status
+
+    assert call(kind=7) == akv.AKV_ERR_INVALID                      # unknown history kind
+    assert call(chunk_tokens=1000) == akv.AKV_ERR_INVALID           # not a multiple of the split
+    assert call(d=96) == akv.AKV_ERR_UNSUPPORTED
+    assert call(Hq=12) == akv.AKV_ERR_INVALID                       # not a multiple of Hkv
+    assert call(kind=akv.AKV_TIER_CODES4, new_row=0x6000) == akv.AKV_ERR_INVALID  # compact histories take no row
+    assert call(n_slots=0) == akv.AKV_ERR_BUDGET                    # 1 split needed
+    assert call(n_tokens=-1) == akv.AKV_ERR_INVALID
+    assert call(o=None) == akv.AKV_ERR_INVALID
+    bad_window = akv.Tier(akv.AKV_TIER_CODES4, 0x1000, 0x2000, lens=[16])
+    assert call(window=bad_window) == akv.AKV_ERR_INVALID          # the window is exact BF16
+    st.destroy()
+
+
+def test_aging_create_refusals(akv):
+    """akv_aging_create checks the description on the host; nothing touches the device."""
+    B, H, d, W = 2, 8, 128, 64
+    R = W // 16 + 2
+    win = akv.Tier(akv.AKV_TIER_BF16, 0x10000, 0x20000, lens=[0] * B, paged=True, page_table=0x30000,
+                   page_table_stride=R, n_pages=B * R, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
+    cmp = akv.Tier(akv.AKV_TIER_CODES4, 0x40000, 0x50000, lens=[0] * B, paged=True, page_table=0x60000,
+                   page_table_stride=8, n_pages=16, stride_seq=H, stride_head=1)
+    good = dict(B=B, Hq=32, Hkv=H, d=d, split_tokens=512, softmax_scale=0.1, window_tokens=W, ring_pages=R,
+                window=win, compact=cmp, compact_len=[32, 0], window_len=[W, W + 5], ring_head=[0, 1],
+                page_lists=[[3, 4, 5], [6]], lists_dev=0x70000, o_part=0x80000, lse_part=0x90000, n_slots=64)
+
+    def refused(**kw):
+        args = dict(good)
+        args.update(kw)
+        with pytest.raises(akv.AkvError) as e:
+            akv.Aging(**args)
+        return e.value.status
+
+    ctx = akv.Aging(**good)
+    c, w, r, aged = ctx.state()
+    assert list(c) == [32, 0] and list(w) == [W, W + 5] and list(r) == [0, 1] and aged == 0
+    ctx.destroy()
+    assert refused(window_tokens=40) == akv.AKV_ERR_INVALID          # not a multiple of 16
+    assert refused(ring_pages=R - 1) == akv.AKV_ERR_INVALID          # the ring cannot hold W + 16 tokens
+    assert refused(window_len=[W - 1, W]) == akv.AKV_ERR_INVALID     # a window below W
+    assert refused(compact_len=[40, 0]) == akv.AKV_ERR_INVALID       # not a whole code page
+    assert refused(page_lists=[[3], [6]]) == akv.AKV_ERR_INVALID     # fewer pages than the compact tokens use
+    assert refused(ring_head=[0, R]) == akv.AKV_ERR_INVALID
+    assert refused(d=80) == akv.AKV_ERR_UNSUPPORTED
+    assert refused(window=cmp) == akv.AKV_ERR_INVALID
