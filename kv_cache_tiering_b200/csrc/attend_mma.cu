@@ -443,13 +443,26 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
   __syncwarp();
   wait_prior_grids();  // every global access comes after this
 
+  // paged tiers: lane j holds the page ids of steps j and 32 + j of item pid_slot (one
+  // coalesced load per lane when the loader reaches an item)
+  int pid0 = 0, pid1 = 0, pid_slot = -1;
   // lane 0 fills stage st with step s of item it: one TMA box per 64-element half of K and V
   auto load_step = [&](const Item& it, int s, int st) {
+    int page = 0;
+    if (p.tier.paged) {  // warp-uniform
+      if (it.slot != pid_slot) {
+        pid_slot = it.slot;
+        const int nst = (it.n + 15) >> 4, lp0 = it.t0 >> 4;
+        pid0 = lane < nst ? (int)tier_page(p.tier, it.b, lp0 + lane, p.err) : 0;
+        pid1 = 32 + lane < nst ? (int)tier_page(p.tier, it.b, lp0 + 32 + lane, p.err) : 0;
+      }
+      page = __shfl_sync(kFull, s < 32 ? pid0 : pid1, s & 31);
+    }
     if (lane == 0) {
       int c1, c3;
       if (p.tier.paged) {
         c1 = 0;
-        c3 = (int)tier_page(p.tier, it.b, (it.t0 + 16 * s) >> 4, p.err);
+        c3 = page;
       } else {
         c1 = it.t0 + 16 * s;
         c3 = it.b;
@@ -727,7 +740,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   constexpr int CH = C::BLOCK / 16;  // 16-byte chunks per block
   static_assert(CH > 32 && CH <= 96, "at most three chunk rounds per block");
   int ld_item = lo, ld_left = 0;  // the loader's item and its steps not yet issued
-  int ld_b = 0, ld_lp = 0;         // its sequence and the logical page of its next step
+  int ld_step = 0;                 // the step of that item the loader issues next
+  // paged tiers: lane j holds the page ids of the item's steps j and 32 + j, loaded (one
+  // coalesced load per lane) when the loader reaches the item, so issuing a step needs a
+  // shuffle instead of a dependent global load
+  int ld_pid0 = 0, ld_pid1 = 0;
   // contiguous tiers: this lane's first chunk of the next key block, stepped by one token
   // block per step; paged tiers: of the head's block in page 0.  A value block sits at a
   // fixed distance from its key block.
@@ -738,16 +755,22 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   auto ld_begin = [&]() {
     const Item it = item_at(p, ld_item);
     ld_left = (it.n + 15) >> 4;
-    ld_b = it.b;
-    ld_lp = it.t0 >> 4;
+    ld_step = 0;
+    const int lp0 = it.t0 >> 4;
     int64_t blk = (int64_t)it.kvh * p.tier.s_head;
-    if (!p.tier.paged) blk += (int64_t)it.b * p.tier.s_seq + (int64_t)ld_lp * p.tier.s_tok;
+    if (p.tier.paged) {
+      ld_pid0 = lane < ld_left ? (int)tier_page(p.tier, it.b, lp0 + lane, p.err) : 0;
+      ld_pid1 = 32 + lane < ld_left ? (int)tier_page(p.tier, it.b, lp0 + 32 + lane, p.err) : 0;
+    } else {
+      blk += (int64_t)it.b * p.tier.s_seq + (int64_t)lp0 * p.tier.s_tok;
+    }
     ld_k = p.tier.k + blk * C::BLOCK + lane16;
   };
   auto ld_issue = [&](uint32_t stage_s) {  // fills the stage at shared address stage_s
     const uint8_t* kb = ld_k;
     if (p.tier.paged) {
-      kb += tier_page(p.tier, ld_b, ld_lp, p.err) * p.tier.s_seq * (int64_t)C::BLOCK;
+      const int64_t page = __shfl_sync(kFull, ld_step < 32 ? ld_pid0 : ld_pid1, ld_step & 31);
+      kb += page * p.tier.s_seq * (int64_t)C::BLOCK;
     } else {
       ld_k += step_bytes;
     }
@@ -763,7 +786,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
       cp_async16(dst + C::K_OFF + 1024, kb + 1024);
       cp_async16(dst + C::V_OFF + 1024, vb + 1024);
     }
-    ++ld_lp;
+    ++ld_step;
     if (--ld_left == 0 && ++ld_item < hi) ld_begin();
   };
   if (busy) {
