@@ -79,16 +79,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
   return false;
 }
+// L2 policy of the K/V streams: every history byte is read once per launch, so its lines
+// are the first to go and the queries, page tables and partial outputs (read again by the
+// merge) stay in L2.  Worth 3-4% on the BF16 tier and about 2% on the compact tier.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));  // pure: may be re-issued
+  return pol;
+}
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                            uint32_t bar) {
+                                            uint32_t bar, uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
-      "[%6];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
       : "memory");
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "l"(pol));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
@@ -446,6 +454,7 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
   // paged tiers: lane j holds the page ids of steps j and 32 + j of item pid_slot (one
   // coalesced load per lane when the loader reaches an item)
   int pid0 = 0, pid1 = 0, pid_slot = -1;
+  const uint64_t pol = l2_evict_first();
   // lane 0 fills stage st with step s of item it: one TMA box per 64-element half of K and V
   auto load_step = [&](const Item& it, int s, int st) {
     int page = 0;
@@ -468,14 +477,16 @@ __global__ void __launch_bounds__(NW * 32, 1) attend_bf16_mma(const __grid_const
         c3 = it.b;
       }
       const uint32_t bar = bar_s + 8 * st, dst = ring_s + st * C::STAGE;
-      const int lc[3] = {c1, it.kvh, c3};
-      const int x1 = lc[p.tperm[0]], x2 = lc[p.tperm[1]], x3 = lc[p.tperm[2]];
+      // TMA dimension j + 1 takes logical coordinate tperm[j] (selects, not an indexed
+      // array, which would live in local memory)
+      auto pick = [&](int j) { return p.tperm[j] == 0 ? c1 : (p.tperm[j] == 1 ? it.kvh : c3); };
+      const int x1 = pick(0), x2 = pick(1), x3 = pick(2);
       fence_proxy_async();
       mbar_expect_tx(bar, C::STAGE);
 #pragma unroll
       for (int hv = 0; hv < C::HALVES; ++hv) {
-        tma_load_4d(dst + hv * C::BOX, &p.tmk, 64 * hv, x1, x2, x3, bar);
-        tma_load_4d(dst + C::TILE + hv * C::BOX, &p.tmv, 64 * hv, x1, x2, x3, bar);
+        tma_load_4d(dst + hv * C::BOX, &p.tmk, 64 * hv, x1, x2, x3, bar, pol);
+        tma_load_4d(dst + C::TILE + hv * C::BOX, &p.tmv, 64 * hv, x1, x2, x3, bar, pol);
       }
     }
   };
@@ -767,6 +778,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     ld_k = p.tier.k + blk * C::BLOCK + lane16;
   };
   auto ld_issue = [&](uint32_t stage_s) {  // fills the stage at shared address stage_s
+    const uint64_t pol = l2_evict_first();
     const uint8_t* kb = ld_k;
     if (p.tier.paged) {
       const int64_t page = __shfl_sync(kFull, ld_step < 32 ? ld_pid0 : ld_pid1, ld_step & 31);
@@ -776,15 +788,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     }
     const uint8_t* vb = kb + kv_delta;
     const uint32_t dst = stage_s + lane16;
-    cp_async16(dst + C::K_OFF, kb);
-    cp_async16(dst + C::V_OFF, vb);
+    cp_async16(dst + C::K_OFF, kb, pol);
+    cp_async16(dst + C::V_OFF, vb, pol);
     if (CH >= 64 || 32 + lane < CH) {
-      cp_async16(dst + C::K_OFF + 512, kb + 512);
-      cp_async16(dst + C::V_OFF + 512, vb + 512);
+      cp_async16(dst + C::K_OFF + 512, kb + 512, pol);
+      cp_async16(dst + C::V_OFF + 512, vb + 512, pol);
     }
     if (64 + lane < CH) {
-      cp_async16(dst + C::K_OFF + 1024, kb + 1024);
-      cp_async16(dst + C::V_OFF + 1024, vb + 1024);
+      cp_async16(dst + C::K_OFF + 1024, kb + 1024, pol);
+      cp_async16(dst + C::V_OFF + 1024, vb + 1024, pol);
     }
     ++ld_step;
     if (--ld_left == 0 && ++ld_item < hi) ld_begin();

@@ -162,6 +162,18 @@ class HybridResident:
         return [self.B * H * 2 * Tc * (d // 2 + 2), self.B * H * 2 * self.W * d * 2]
 
 
+def code_page_pool(n_pages: int, H: int, d: int, device, zero: bool = False):
+    """Paged compact pool ``[P][Hkv][2][block]``: the key block and the value block of one
+    (page, KV head) sit side by side, so a 16-token step reads one 2 x 1056-byte span.  DRAM
+    serves whole 128-byte lines; a 1056-byte block read alone at a random page always spans 9
+    lines (96 B more than it holds), a 2112-byte span 17 (64 B more).
+    Returns (pool, key view, value view, stride_seq, stride_head), the strides in blocks."""
+    bb = akv.codes4_block_bytes(d)
+    alloc = torch.zeros if zero else torch.empty
+    pool = alloc((n_pages, H, 2, bb), dtype=torch.uint8, device=device)
+    return pool, pool[:, :, 0], pool[:, :, 1], 2 * H, 2
+
+
 class RaggedPaged:
     """Ragged paged hybrid batch: per-sequence lengths, 16-token pages drawn from two pools
     through seeded random page permutations; the newest W tokens exact (BF16 pool
@@ -186,15 +198,14 @@ class RaggedPaged:
         n_ex, n_cp = int(ex_pages.sum()), max(1, int(cp_pages.sum()))
         self.ex_k = torch.zeros((n_ex, H, 16, d), dtype=torch.int16, device=device)
         self.ex_v = torch.zeros((n_ex, H, 16, d), dtype=torch.int16, device=device)
-        bb = akv.codes4_block_bytes(d)
-        self.cp_k = torch.empty((n_cp, H, bb), dtype=torch.uint8, device=device)
-        self.cp_v = torch.empty((n_cp, H, bb), dtype=torch.uint8, device=device)
+        self.cp_pool, self.cp_k, self.cp_v, cs, ch = code_page_pool(n_cp, H, d, device)
+        self.cp_strides = dict(stride_seq=cs, stride_head=ch)
         self.ex_table = torch.from_numpy(self.ex_table_np).to(device)
         self.cp_table = torch.from_numpy(self.cp_table_np).to(device)
         self.enc_err = torch.zeros(1, dtype=torch.int32, device=device)
         self.codes_tier = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=cp_len, paged=True,
                                    page_table=self.cp_table, page_table_stride=self.cp_table_np.shape[1],
-                                   n_pages=n_cp, stride_seq=H, stride_head=1)
+                                   n_pages=n_cp, **self.cp_strides)
         self.exact_tier = akv.Tier(akv.AKV_TIER_BF16, self.ex_k, self.ex_v, lens=ex_len, paged=True,
                                    page_table=self.ex_table, page_table_stride=self.ex_table_np.shape[1],
                                    n_pages=n_ex, stride_seq=H * 16 * d, stride_head=16 * d, stride_token=d)
@@ -220,8 +231,7 @@ class RaggedPaged:
                 src = akv.Tier(akv.AKV_TIER_BF16, ks, vs, lens=[c], stride_seq=0, stride_head=c * d, stride_token=d)
                 row = self.cp_table[b:b + 1]
                 dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True, page_table=row,
-                               page_table_stride=self.cp_table_np.shape[1], n_pages=n_cp, stride_seq=H,
-                               stride_head=1)
+                               page_table_stride=self.cp_table_np.shape[1], n_pages=n_cp, **self.cp_strides)
                 akv.akv_encode_history(src, dst, 1, H, d, self.enc_err)
                 torch.cuda.current_stream().synchronize()
                 del ks, vs
@@ -241,7 +251,7 @@ class RaggedPaged:
                 src = akv.Tier(akv.AKV_TIER_BF16, k, v, lens=[c], stride_seq=0, stride_head=L * d, stride_token=d)
                 dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True,
                                page_table=self.cp_table[b:b + 1], page_table_stride=self.cp_table_np.shape[1],
-                               n_pages=n_cp, stride_seq=H, stride_head=1)
+                               n_pages=n_cp, **self.cp_strides)
                 akv.akv_encode_history(src, dst, 1, H, d, self.enc_err)
             e = int(ex_len[b])
             pages = -(-e // 16)
@@ -571,8 +581,8 @@ class AgingHybrid:
         self.ex_table_np = np.array([[b * self.R + j for j in range(self.R)] for b in range(self.B)], np.int32)
         self.ex_k = torch.zeros((self.B * self.R, H, 16, d), dtype=torch.int16, device=device)
         self.ex_v = torch.zeros_like(self.ex_k)
-        self.cp_k = torch.zeros((self.n_cp, H, self.bb), dtype=torch.uint8, device=device)
-        self.cp_v = torch.zeros_like(self.cp_k)
+        self.cp_pool, self.cp_k, self.cp_v, cs, ch = code_page_pool(self.n_cp, H, d, device, zero=True)
+        self.cp_strides = dict(stride_seq=cs, stride_head=ch)
         self.cp_table = torch.from_numpy(self.cp_table_np).to(device)
         self.ex_table = torch.from_numpy(self.ex_table_np).to(device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
@@ -593,7 +603,7 @@ class AgingHybrid:
                 src = akv.Tier(akv.AKV_TIER_BF16, kd, vd, lens=[c], stride_seq=0, stride_head=L * d, stride_token=d)
                 dst = akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=[c], paged=True,
                                page_table=self.cp_table[b:b + 1], page_table_stride=self.cp_table_np.shape[1],
-                               n_pages=self.n_cp, stride_seq=H, stride_head=1)
+                               n_pages=self.n_cp, **self.cp_strides)
                 akv.akv_encode_history(src, dst, 1, H, d, self.err)
             w = L - c
             pages = -(-w // 16)
@@ -618,7 +628,7 @@ class AgingHybrid:
                              akv.Tier(akv.AKV_TIER_CODES4, self.cp_k, self.cp_v, lens=self.c.astype(np.int32),
                                       paged=True, page_table=self.cp_table,
                                       page_table_stride=self.cp_table_np.shape[1], n_pages=self.n_cp,
-                                      stride_seq=H, stride_head=1),
+                                      **self.cp_strides),
                              self.c.astype(np.int32), self.win.astype(np.int32), self.ring0.astype(np.int32),
                              self.owned, self._enc_dev, self.o_part, self.lse_part, self.o_part.shape[0])
         self._aged0 = int(self.c.sum() // 16)
