@@ -44,7 +44,7 @@ METRIC = "decode-attention history tokens/s/GPU & achieved HBM GB/s vs B200 peak
 UNIT = "history tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 WORKLOADS = ["ragged", "exact", "hybrid", "tiny", "staged", "staged-hybrid", "aging"]
-PER_CONFIG = ("exact", "hybrid", "staged", "staged-hybrid")
+PER_CONFIG = ("exact", "hybrid", "staged", "staged-hybrid", "aging")
 STAGED = ("staged", "staged-hybrid")
 
 
@@ -826,6 +826,8 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
     variant = variant_of(args.variant)
     inputs = [st.inputs(i) for i in range(n_steps)]
     stream = torch.cuda.current_stream()
+    sampler = ClockSampler(ctx.local)
+    sampler.start()
     for i in range(n_warm):
         st.step(*inputs[i], variant, stream)
     torch.cuda.synchronize()
@@ -833,11 +835,14 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
     tok0 = int(st.c.sum() + st.win.sum())  # history tokens before the first timed step
     ctx.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tw0 = time.monotonic()
     e0.record(stream)
     for i in range(n_warm, n_steps):
         st.step(*inputs[i], variant, stream, sync_state=False)
     e1.record(stream)
     torch.cuda.synchronize()
+    tw1 = time.monotonic()
+    sampler.stop()
     ms = ctx.max(e0.elapsed_time(e1))
     st._state()
     aged = st.aged_blocks - aged0
@@ -856,7 +861,8 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
                        "step": "one akv_aging_step call (append, aging encode, attention launches, merge)"},
             "aged_pages_in_timed_steps": int(aged),
             "e2e": None, "gpu_launches": steps * 4 + 2 * int(aged > 0) * (aged // wl.B),
-            "device_error_word": err}
+            # the timed steps take milliseconds: the samples within 0.25 s of them
+            "clocks": sampler.summary(tw0 - 0.25, tw1 + 0.25), "device_error_word": err}
 
 
 def run_workload(name, ctx, args, steps, warmup, cpu_s):

@@ -448,8 +448,9 @@ akv_status akv_staged_decode(akv_stager* stager, const akv_staged_history* hist,
  * that page in the compact page table and rotates its window page-table row (both written
  * on the device by the call) -- then attends both tiers with the standard slot layout
  * (akv_plan_slots) into o_part / lse_part (n_slots slots) and merges into o, lse (device
- * float32 [B][Hq][d], [B][Hq]).  Everything is enqueued on `stream`; the context keeps the
- * lengths on the host.  lists_dev: device int32 scratch of 2 B entries (the encode's page
+ * float32 [B][Hq][d], [B][Hq]).  Everything is enqueued on `stream` (on a step that ages
+ * no page the append may run on the library's side stream just before the window's launch,
+ * joined back to `stream` like that launch); the context keeps the lengths on the host.  lists_dev: device int32 scratch of 2 B entries (the encode's page
  * lists).  A sequence with no code page left is refused (AKV_ERR_BUDGET) before anything is
  * enqueued.  The tiers' lens and slot_base are ignored.  Results equal the same calls made
  * one by one.  akv_aging_state reads the current lengths, ring heads and the number of pages

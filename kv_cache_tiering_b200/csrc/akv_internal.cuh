@@ -256,11 +256,25 @@ struct WorkspaceLayout {
 };
 WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t n_slots);
 
+// A checked token append of at most kMaxSeqPerLaunch sequences, not yet enqueued.
+struct PendingAppend {
+  AppendParams p;
+  int d, n_seq;
+  bool write;  // some position is >= 0 (false: nothing to enqueue)
+};
+// The checks and parameters of akv_append_tokens (same refusals); *single is false when the
+// batch needs more than one launch, and then `out` is not filled.
+akv_status prepare_append(const akv_tier* tier, const int32_t* pos, int B, int Hkv, int d, const void* new_k,
+                          const void* new_v, int32_t* err_word, PendingAppend* out, bool* single);
+
 // Validated split attention of every tier; copy_in (may be null) is enqueued after the checks
-// and before the first attention launch.
+// and before the first attention launch.  append (may be null) writes a token the BF16 tier
+// reads: it is enqueued before that tier's launch, on the stream that launch goes to, so when
+// the tiers run side by side the append overlaps the compact tier.
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in = nullptr);
+                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in = nullptr,
+                       const PendingAppend* append = nullptr);
 
 // Set the thread's last-error message; returns st.
 akv_status set_error(akv_status st, const char* msg);

@@ -267,6 +267,36 @@ akv_status akv_plan_slots(int B, int n_tiers, const int32_t* const* tier_lens, i
 
 akv_status akv_append_tokens(const akv_tier* tier, const int32_t* pos, int B, int Hkv, int d, const void* new_k,
                              const void* new_v, int32_t* err_word, akv_stream_t stream) {
+  akv::PendingAppend one;
+  bool single = false;
+  akv_status s = akv::prepare_append(tier, pos, B, Hkv, d, new_k, new_v, err_word, &one, &single);
+  if (s != AKV_OK || !one.write) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (single) {
+    const cudaError_t e = akv::launch_append(one.p, d, one.n_seq, st);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "append launch");
+  }
+  akv::AppendParams p = one.p;
+  for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
+    const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
+    p.b0 = b0;
+    for (int i = 0; i < n; ++i) p.pos[i] = pos[b0 + i];
+    cudaError_t e = akv::launch_append(p, d, n, st);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  return ok();
+}
+
+}  // extern "C"
+
+namespace akv {
+
+akv_status prepare_append(const akv_tier* tier, const int32_t* pos, int B, int Hkv, int d, const void* new_k,
+                          const void* new_v, int32_t* err_word, PendingAppend* out, bool* single) {
+  *single = B <= akv::kMaxSeqPerLaunch;
+  out->d = d;
+  out->n_seq = 0;
+  out->write = false;
   if (B < 0 || Hkv <= 0) return fail(AKV_ERR_INVALID, "B must be >= 0 and Hkv > 0");
   if (d != 64 && d != 128) return fail(AKV_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
   if (Hkv > 65535) return fail(AKV_ERR_UNSUPPORTED, "Hkv %d too large", Hkv);
@@ -283,7 +313,7 @@ akv_status akv_append_tokens(const akv_tier* tier, const int32_t* pos, int B, in
     lens[b] = pos[b] < 0 ? 0 : pos[b] + 1;
     any |= pos[b] >= 0;
   }
-  if (!any) return ok();
+  if (!any) return ok();  // nothing to write: n_seq stays 0
   if (!new_k || !new_v || !aligned(new_k, 16) || !aligned(new_v, 16))
     return fail(AKV_ERR_INVALID, "new_k and new_v must be 16-byte aligned device pointers");
   akv_tier view = *tier;
@@ -297,16 +327,20 @@ akv_status akv_append_tokens(const akv_tier* tier, const int32_t* pos, int B, in
   p.new_v = static_cast<const uint16_t*>(new_v);
   p.err = err_word;
   p.Hkv = Hkv;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int b0 = 0; b0 < B; b0 += akv::kMaxSeqPerLaunch) {
-    const int n = std::min(akv::kMaxSeqPerLaunch, B - b0);
-    p.b0 = b0;
-    for (int i = 0; i < n; ++i) p.pos[i] = pos[b0 + i];
-    cudaError_t e = akv::launch_append(p, d, n, st);
-    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  p.b0 = 0;
+  out->p = p;
+  out->write = true;
+  if (*single) {
+    for (int i = 0; i < B; ++i) out->p.pos[i] = pos[i];
+    out->n_seq = B;
   }
   return ok();
 }
+
+}  // namespace akv
+
+extern "C" {
+
 
 akv_status akv_encode_history(const akv_tier* src, const akv_tier* dst, int B, int Hkv, int d, int32_t* err_word,
                               akv_stream_t stream) {
@@ -441,15 +475,24 @@ bool stream_on_current_device(cudaStream_t st) {
   return cur == dev;
 }
 
+akv_status enqueue_append(const akv::PendingAppend& a, cudaStream_t st) {
+  const cudaError_t e = akv::launch_append(a.p, a.d, a.n_seq, st);
+  return e == cudaSuccess ? AKV_OK : cuda_fail(e, "append launch");
+}
+
+// x (the BF16 tier, after `append` when given) on the side stream, c (the compact tier) on st
 akv_status side_by_side(const PlannedLaunch& c, const PlannedLaunch& x, int share, int rest, int d, int G,
-                        cudaStream_t st) {
+                        cudaStream_t st, const akv::PendingAppend* append) {
   std::lock_guard<std::mutex> lock(side_mutex());
   SideLane* lane = nullptr;
   cudaError_t e = side_lane(lane);
   if (e != cudaSuccess) return cuda_fail(e, "side stream");
   if ((e = cudaEventRecord(lane->fork, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = cudaStreamWaitEvent(lane->stream, lane->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
-  const cudaError_t ex = akv::launch_attend_mma(x.p, d, G, x.kind, x.items, lane->stream, rest, false);
+  cudaError_t ex = append ? akv::launch_append(append->p, append->d, append->n_seq, lane->stream) : cudaSuccess;
+  // after an append on the same stream the launch overlaps it (the kernel waits for the
+  // append's writes before its first global read)
+  if (ex == cudaSuccess) ex = akv::launch_attend_mma(x.p, d, G, x.kind, x.items, lane->stream, rest, append != nullptr);
   // the join is recorded and waited for even after a failed launch, so `st` never runs ahead of
   // anything the side stream was given
   if ((e = cudaEventRecord(lane->join, lane->stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -473,7 +516,8 @@ namespace akv {
 
 akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softmax_scale, const akv_tier* tiers,
                        int n_tiers, int split_tokens, float* o_part, float* lse_part, int64_t n_slots, int variant,
-                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in) {
+                       int32_t* err_word, cudaStream_t st, const CopyIn* copy_in, const PendingAppend* append) {
+  if (append && (!append->write || append->n_seq <= 0)) append = nullptr;
   if (B < 0 || n_tiers < 0) return fail(AKV_ERR_INVALID, "negative B or n_tiers");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return fail(AKV_ERR_INVALID, "Hq must be a positive multiple of Hkv");
   const int G = Hq / Hkv;
@@ -494,7 +538,7 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
     if (s != AKV_OK) return s;
     for (int b = 0; b < B; ++b) any |= tiers[i].lens[b] > 0;
   }
-  if (!any) return ok();
+  if (!any) return append ? enqueue_append(*append, st) : ok();
   if (!q || !aligned(q, 16)) return fail(AKV_ERR_INVALID, "q must be a 16-byte aligned device pointer");
   if (!o_part || !lse_part) return fail(AKV_ERR_INVALID, "o_part and lse_part must not be null");
   if (!aligned(o_part, 16)) return fail(AKV_ERR_INVALID, "o_part must be 16-byte aligned");
@@ -543,6 +587,11 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
             if (cs != AKV_OK) return cs;
             copy_in = nullptr;
           }
+          if (append) {
+            const akv_status as = enqueue_append(*append, st);
+            if (as != AKV_OK) return as;
+            append = nullptr;
+          }
           // AUTO takes the tensor-core path, which measures faster on both tiers
           cudaError_t e = simt ? akv::launch_attend_simt(p, d, G, tiers[i].kind, (int)items, st)
                                : akv::launch_attend_mma(p, d, G, tiers[i].kind, (int)items, st);
@@ -563,7 +612,11 @@ akv_status attend_impl(const void* q, int B, int Hq, int Hkv, int d, float softm
     const PlannedLaunch& x = two[0].kind == AKV_TIER_CODES4 ? two[1] : two[0];
     const int share = compact_sm_share(sms, c.items, akv::codes_warps_per_cta(G), ceil_div(c.split_len, 16), x.items,
                                        ceil_div(ceil_div(x.split_len, 16), 8));
-    if (share > 0) return side_by_side(c, x, share, sms - share, d, G, st);
+    if (share > 0) return side_by_side(c, x, share, sms - share, d, G, st, append);
+  }
+  if (append) {
+    const akv_status as = enqueue_append(*append, st);
+    if (as != AKV_OK) return as;
   }
   for (int k = 0; k < n_launch; ++k) {
     const PlannedLaunch& l = two[k];

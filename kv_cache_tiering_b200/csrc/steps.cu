@@ -230,12 +230,24 @@ extern "C" akv_status akv_aging_step(akv_aging* g, const void* q, const void* k_
   for (int b = 0; b < B; ++b)
     if (g->win[b] + 1 >= a.window_tokens + 16 && g->c[b] / 16 >= (int32_t)g->pages[b].size())
       return refuse(AKV_ERR_BUDGET, "sequence %d has no code page left to age into", b);
-  // 1. the new token goes to position win[b] of the window
+  // 1. the new token goes to position win[b] of the window.  A step that ages a page
+  // enqueues the append first (the aging rewrites the window's page table); otherwise the
+  // append is handed to the attention call, which runs it just before the window's launch
+  // (beside the compact tier when the two tiers share the GPU).
   for (int b = 0; b < B; ++b) g->pos[b] = g->win[b];
+  bool ages = false;
+  for (int b = 0; b < B; ++b) ages |= g->win[b] + 1 >= a.window_tokens + 16;
   akv_tier wt = g->window;
   wt.lens = g->win.data();
-  akv_status st = akv_append_tokens(&wt, g->pos.data(), B, a.Hkv, a.d, k_new, v_new, err_word, stream);
+  akv::PendingAppend app;
+  bool single = false;
+  akv_status st = akv::prepare_append(&wt, g->pos.data(), B, a.Hkv, a.d, k_new, v_new, err_word, &app, &single);
   if (st != AKV_OK) return st;
+  const bool deferred = single && !ages;
+  if (!deferred) {
+    st = akv_append_tokens(&wt, g->pos.data(), B, a.Hkv, a.d, k_new, v_new, err_word, stream);
+    if (st != AKV_OK) return st;
+  }
   // 2. a window of W + 16 tokens hands its oldest page to the compact tier
   std::vector<int> aging;
   for (int b = 0; b < B; ++b) {
@@ -290,9 +302,14 @@ extern "C" akv_status akv_aging_step(akv_aging* g, const void* q, const void* k_
   tiers[0].slot_base = g->cbase.data();
   tiers[1].lens = g->win.data();
   tiers[1].slot_base = g->wbase.data();
-  st = akv_decode_attend(q, B, a.Hq, a.Hkv, a.d, a.softmax_scale, tiers, 2, a.split_tokens, a.o_part, a.lse_part,
-                         a.n_slots, variant, err_word, stream);
-  if (st != AKV_OK) return st;
+  st = akv::attend_impl(q, B, a.Hq, a.Hkv, a.d, a.softmax_scale, tiers, 2, a.split_tokens, a.o_part, a.lse_part,
+                        a.n_slots, variant, err_word, s, nullptr, deferred ? &app : nullptr);
+  if (st != AKV_OK) {
+    // the window now counts the new token: write it even though the step fails (writing it
+    // twice stores the same row)
+    if (deferred) akv_append_tokens(&wt, g->pos.data(), B, a.Hkv, a.d, k_new, v_new, err_word, stream);
+    return st;
+  }
   st = akv_merge_lse(a.o_part, a.lse_part, a.n_slots, g->seq_base.data(), g->seq_n.data(), B, a.Hq, a.d, o, lse,
                      stream);
   if (st != AKV_OK) return st;
