@@ -642,13 +642,20 @@ def run_resident(name, ctx, args, steps, warmup, cpu_s):
     return line
 
 
-def pcie_ceiling(chunk_bytes: int, device, rounds: int = 5, copies: int = 32) -> float:
+def pcie_ceiling(chunk_bytes: int, device, sources, rounds: int = 5, copies: int = 32) -> float:
     """Pinned host-to-device bandwidth (GB/s) with the copies the stager issues: chunk_bytes
-    copies from consecutive spans of a pinned buffer into two alternating device buffers, back
-    to back on one stream; host wall clock between timing-disabled fences, best of `rounds`."""
+    spans of the staged run's own pinned history (`sources`, its per-layer host tensors, so
+    the same pages and NUMA placement) into two alternating device buffers, back to back on
+    one stream; host wall clock between timing-disabled fences, best of `rounds`."""
     import torch
-    span = copies * chunk_bytes
-    src = torch.empty(span, dtype=torch.uint8).pin_memory()
+    spans = []
+    for h in sources:
+        flat = h.view(torch.uint8).reshape(-1)
+        for c in range(flat.numel() // chunk_bytes):
+            if len(spans) < copies:
+                spans.append(flat[c * chunk_bytes:(c + 1) * chunk_bytes])
+    if not spans:
+        return 0.0
     dst = [torch.empty(chunk_bytes, dtype=torch.uint8, device=device) for _ in range(2)]
     s = torch.cuda.Stream(device)
     fence = torch.cuda.Event()  # timing disabled: it does not serialise the copies it follows
@@ -657,14 +664,14 @@ def pcie_ceiling(chunk_bytes: int, device, rounds: int = 5, copies: int = 32) ->
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         with torch.cuda.stream(s):
-            for c in range(copies):
-                dst[c % 2].copy_(src[c * chunk_bytes:(c + 1) * chunk_bytes], non_blocking=True)
+            for c, src in enumerate(spans):
+                dst[c % 2].copy_(src, non_blocking=True)
             fence.record(s)
         fence.synchronize()
         dt = time.perf_counter() - t0
         if r > 0:  # the first round warms the path
-            best = max(best, span / dt / 1e9)
-    del src, dst
+            best = max(best, len(spans) * chunk_bytes / dt / 1e9)
+    del dst
     return best
 
 
@@ -747,7 +754,7 @@ def run_staged(name, ctx, args, steps, warmup, cpu_s):
             o_host.copy_(st.o, non_blocking=True)
             lse_host.copy_(st.lse, non_blocking=True)
 
-    pcie_peak = pcie_ceiling(chunk_bytes, dev)
+    pcie_peak = pcie_ceiling(chunk_bytes, dev, st.host)
     sampler = ClockSampler(ctx.local)
     sampler.start()
     for i in range(n_warm):
