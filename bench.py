@@ -829,12 +829,12 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
     T, W = wl.extra["T"], wl.extra["window"]
     n_warm = max(3, warmup)
     n_steps = n_warm + steps
+    sampler = ClockSampler(ctx.local)  # started early: its first sample takes a moment
+    sampler.start()
     st = workloads.AgingHybrid(wl, dev, [T] * wl.B, W, max_steps=n_steps + 1, source="torch")
     variant = variant_of(args.variant)
     inputs = [st.inputs(i) for i in range(n_steps)]
     stream = torch.cuda.current_stream()
-    sampler = ClockSampler(ctx.local)
-    sampler.start()
     for i in range(n_warm):
         st.step(*inputs[i], variant, stream)
     torch.cuda.synchronize()
