@@ -89,3 +89,35 @@ def test_append_tokens_contiguous_paged_and_bounds(mods, cuda):
     assert np.array_equal(pkk[1, :, 1], new_k[0]) and np.array_equal(pkk[0, :, 2], new_k[1])
     assert np.count_nonzero(pkk[2]) == 0 and np.count_nonzero(pkk[3]) == 0   # nothing written for sequence 2
     assert int(err.item()) & akv.AKV_EFLAG_BOUNDS
+
+
+def test_aging_step_at_hybrid_shape_equals_separate_calls(mods, cuda):
+    """At the hybrid shape (batch 4 x 32768, W = 2048) the two tiers share the GPU, and a step
+    that ages no page runs its append on the window's stream just before the window's launch,
+    beside the compact tier.  After every step the same attention and merge, enqueued as
+    separate calls on the state the step left (the appended token included), give the step's
+    output bit for bit.  20 steps include one aging step (the window reaches W + 16 at step
+    16)."""
+    import torch
+    akv, workloads = mods
+    base = synth.WORKLOADS["hybrid"]
+    wl = synth.Workload("aging-hybrid-shape", base.B, base.Hq, base.Hkv, base.d, base.split_tokens, seed=base.seed,
+                        extra=dict(base.extra))
+    T, W = wl.extra["T"], wl.extra["window"]
+    steps = 20
+    st = workloads.AgingHybrid(wl, cuda, [T] * wl.B, W, max_steps=steps + 2, source="torch")
+    aged0 = st.aged_blocks
+    for s in range(steps):
+        q, kn, vn = st.inputs(s)
+        st.step(q, kn, vn)
+        torch.cuda.synchronize()
+        compact = akv.Tier(akv.AKV_TIER_CODES4, st.cp_k, st.cp_v, lens=st.c.astype(np.int32), paged=True,
+                           page_table=st.cp_table, page_table_stride=st.cp_table_np.shape[1], n_pages=st.n_cp,
+                           **st.cp_strides)
+        ref = workloads.DecodeStep(st.B, wl.Hq, wl.Hkv, wl.d, wl.split_tokens, wl.scale,
+                                   [compact, st._exact_tier(lens=st.win.astype(np.int32))], cuda)
+        ref.step(q)
+        torch.cuda.synchronize()
+        assert torch.equal(ref.o, st.o) and torch.equal(ref.lse, st.lse), s
+        assert int(st.err.item()) == 0 and int(ref.err.item()) == 0
+    assert st.aged_blocks - aged0 == wl.B
