@@ -376,29 +376,38 @@ __device__ __forceinline__ void chain_to_smem(float (&acc)[D / 16][4], float m_r
     }
 }
 
-// Unnormalised Walsh-Hadamard transform of a 32*P-vector held P per lane (lane l holds
-// elements [P*l, P*l + P)), Sylvester order.
-template <int P>
-__device__ __forceinline__ void warp_fwht(float (&x)[P]) {
-  const int lane = threadIdx.x & 31;
+// Unnormalised Walsh-Hadamard transform, Sylvester order, of a (C * L)-vector held by a
+// group of L consecutive lanes, C elements per lane: lane `part` of the group holds elements
+// [C part, C part + C).  The stages run in increasing stride: those below C inside the lane,
+// the others against lane part ^ (stride / C) of the same group.  Every butterfly is
+// (lower + upper, lower - upper), so the result does not depend on C.
+template <int C, int L>
+__device__ __forceinline__ void group_fwht(float (&x)[C], int part) {
 #pragma unroll
-  for (int h = 1; h < P; h <<= 1)
+  for (int h = 1; h < C; h <<= 1)
 #pragma unroll
-    for (int j = 0; j < P; ++j)
+    for (int j = 0; j < C; ++j)
       if ((j & h) == 0) {
         const float a = x[j], b = x[j + h];
         x[j] = a + b;
         x[j + h] = a - b;
       }
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+  for (int m = 1; m < L; m <<= 1) {
+    const bool upper = (part & m) != 0;
 #pragma unroll
-    for (int j = 0; j < P; ++j) {
+    for (int j = 0; j < C; ++j) {
       const float o = __shfl_xor_sync(kFull, x[j], m);
       x[j] = upper ? o - x[j] : x[j] + o;
     }
   }
+}
+
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};\n" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
 // Merge the NW chain states of a finished item (group threads) and write its partials.
@@ -719,9 +728,12 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   using C = CodesCfg<D, G, NWARP, NST>;
   constexpr int DPT = D / 8;                      // value dims per lane group
   constexpr int KB = D / 8;                       // key code bytes per lane
-  constexpr int P = D / 32;                       // coordinates per lane in a warp-wide row
+  // rotations (query in, output out): lane group qh of LPH lanes holds head qh, CPL
+  // coordinates per lane, so the transform needs log2(LPH) shuffle stages, not 5
+  constexpr int LPH = 32 / G, CPL = D / LPH;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const int qh = lane / LPH, qp = lane % LPH;  // this lane's head and part in the rotations
   const uint32_t base_s = smem_u32(smem);
   uint32_t lut_s, ring_s;
   allow_next_grid();
@@ -748,20 +760,23 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   const int lo = gw * q0 + min(gw, r0), hi = lo + q0 + (gw < r0 ? 1 : 0);
   const bool busy = lo < hi;
 
-  // the query rows of an item's G heads, P bf16 coordinates per lane each, one load per head;
-  // the first item's are requested before anything else so their latency hides behind the
-  // stage loads and the table build
-  auto load_q = [&](const Item& it, uint32_t (&qw)[G][P / 2]) {
+  // the query coordinates [CPL qp, CPL qp + CPL) of head qh, as bf16 pairs; the first item's
+  // are requested before anything else so their latency hides behind the stage loads and
+  // the table build
+  auto load_q = [&](const Item& it, uint32_t (&qw)[CPL / 2]) {
+    const uint16_t* qrow = p.q + ((size_t)it.b * p.Hq + (size_t)it.kvh * G + qh) * D + CPL * qp;
+    if constexpr (CPL >= 8) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint16_t* qrow = p.q + ((size_t)it.b * p.Hq + (size_t)it.kvh * G + h) * D + P * lane;
-      if constexpr (P == 4) {
-        const uint2 v = *reinterpret_cast<const uint2*>(qrow);
-        qw[h][0] = v.x;
-        qw[h][1] = v.y;
-      } else {
-        qw[h][0] = *reinterpret_cast<const uint32_t*>(qrow);
+      for (int i = 0; i < CPL / 8; ++i) {
+        const uint4 v = reinterpret_cast<const uint4*>(qrow)[i];
+        qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
       }
+    } else if constexpr (CPL == 4) {
+      const uint2 v = *reinterpret_cast<const uint2*>(qrow);
+      qw[0] = v.x;
+      qw[1] = v.y;
+    } else {
+      qw[0] = *reinterpret_cast<const uint32_t*>(qrow);
     }
   };
   // the lookup table is built from the launch parameters, before the wait for the previous
@@ -779,7 +794,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
   fill_seq_smem(p, &ss_tab);
   const SeqSmem* ss = nullptr;
   wait_prior_grids();
-  uint32_t qw[G][P / 2];
+  uint32_t qw[CPL / 2];
   if (busy) load_q(item_at(p, lo, nullptr), qw);
 
   // ---- loader: the (item, step) of the next stage to fill.  Global step S of this warp
@@ -927,47 +942,44 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
     if (it.pair != q_pair) {
       if (item != lo) load_q(it, qw);
       q_pair = it.pair;
-      // rotate the heads together: H q by shuffles, a power-of-two scale to [0.5, 1), then
-      // the FP16 (high, residual) words of dims (P*lane + j, P*lane + j + 1) into the scratch
-      float x[G][P];
+      // rotate: lane group qh transforms head qh (the tier's rotation signs first), scales it
+      // by a power of two to [0.5, 1) and writes the FP16 (high, residual) words of its dims
+      // (2i, 2i + 1) to scratch words qh D + 2i and qh D + 2i + 1
+      float x[CPL];
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int j = 0; j < P / 2; ++j) {  // the tier's rotation signs come first
-          x[h][2 * j] = bf16lo(qw[h][j]) * coord_sign(p.tier, P * lane + 2 * j);
-          x[h][2 * j + 1] = bf16hi(qw[h][j]) * coord_sign(p.tier, P * lane + 2 * j + 1);
-        }
-#pragma unroll
-      for (int h = 0; h < G; ++h) warp_fwht<P>(x[h]);
-      float mx[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        mx[h] = 0.f;
-#pragma unroll
-        for (int j = 0; j < P; ++j) mx[h] = fmaxf(mx[h], fabsf(x[h][j]));
+      for (int j = 0; j < CPL / 2; ++j) {
+        x[2 * j] = bf16lo(qw[j]) * coord_sign(p.tier, CPL * qp + 2 * j);
+        x[2 * j + 1] = bf16hi(qw[j]) * coord_sign(p.tier, CPL * qp + 2 * j + 1);
       }
+      group_fwht<CPL, LPH>(x, qp);
+      float mx = 0.f;
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1)
+      for (int j = 0; j < CPL; ++j) mx = fmaxf(mx, fabsf(x[j]));
 #pragma unroll
-        for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], off));
+      for (int m = 1; m < LPH; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
       __syncwarp();  // earlier reads of the scratch are done
-      int eA = 0, eB = 0;
+      int e = 0;
+      if (mx > 0.f) frexpf(mx, &e);
+      const float inv = ldexpf(1.f, -e);
+      uint32_t wq[CPL];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        int e = 0;
-        if (mx[h] > 0.f) frexpf(mx[h], &e);
-        const float inv = ldexpf(1.f, -e);
-#pragma unroll
-        for (int j = 0; j < P; j += 2) {
-          const float x0 = x[h][j] * inv, x1 = x[h][j + 1] * inv;
-          const uint32_t hw = pack_f16(x0, x1);
-          const float2 hv = unpack_f16(hw);
-          sts32(scr(h * D + P * lane + j), hw);
-          sts32(scr(h * D + P * lane + j + 1), pack_f16(x0 - hv.x, x1 - hv.y));
-        }
-        if (h == hA) eA = e;
-        if (h == hB) eB = e;
+      for (int j = 0; j < CPL; j += 2) {
+        const float x0 = x[j] * inv, x1 = x[j + 1] * inv;
+        wq[j] = pack_f16(x0, x1);
+        const float2 hv = unpack_f16(wq[j]);
+        wq[j + 1] = pack_f16(x0 - hv.x, x1 - hv.y);
       }
+      if constexpr (CPL >= 4) {
+#pragma unroll
+        for (int j = 0; j < CPL; j += 4) sts128(scr(qh * D + CPL * qp + j), wq[j], wq[j + 1], wq[j + 2], wq[j + 3]);
+      } else {
+        sts64(scr(qh * D + CPL * qp), wq[0], wq[1]);
+      }
+      // the scale exponents of this lane's score heads hA, hB (heads >= G give 0; their
+      // columns are never stored)
+      const int eA_src = hA < G ? hA : 0, eB_src = hB < G ? hB : 0;
+      const int eA_g = __shfl_sync(kFull, e, eA_src * LPH), eB_g = __shfl_sync(kFull, e, eB_src * LPH);
+      const int eA = hA < G ? eA_g : 0, eB = hB < G ? eB_g : 0;
       __syncwarp();
       // column g, step kc: dims 2*KB*tq + 4kc + {0, 1} (b0) and + {2, 3} (b1) of the lane's
       // k range; the scratch holds (high, residual) word pairs per two dims
@@ -1143,23 +1155,26 @@ __global__ void __launch_bounds__(NWARP * 32, 1) attend_codes_mma(const __grid_c
         if (h < G) sts32(scr(h * D + dim), __float_as_uint(acc[mt][e] * ((e & 1) ? f_odd : f_even)));
       }
     __syncwarp();
+    {  // lane group qh rotates head qh back and stores it
+      float x[CPL];
+      if constexpr (CPL >= 4) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float x[P];
-      if constexpr (P == 4) {
-        const uint4 v = lds128<0>(scr(h * D + P * lane));
-        x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
-        x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+        for (int j = 0; j < CPL; j += 4) {
+          const uint4 v = lds128<0>(scr(qh * D + CPL * qp + j));
+          x[j] = __uint_as_float(v.x); x[j + 1] = __uint_as_float(v.y);
+          x[j + 2] = __uint_as_float(v.z); x[j + 3] = __uint_as_float(v.w);
+        }
       } else {
-        const uint2 v = lds64<0>(scr(h * D + P * lane));
+        const uint2 v = lds64<0>(scr(qh * D + CPL * qp));
         x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
       }
-      warp_fwht<P>(x);
+      group_fwht<CPL, LPH>(x, qp);
 #pragma unroll
-      for (int j = 0; j < P; ++j) x[j] *= coord_sign(p.tier, P * lane + j);  // undo the rotation signs
-      float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + h) * D + P * lane;
-      if constexpr (P == 4) {
-        *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+      for (int j = 0; j < CPL; ++j) x[j] *= coord_sign(p.tier, CPL * qp + j);  // undo the rotation signs
+      float* dst = p.o_part + ((size_t)it.slot * p.Hq + it.kvh * G + qh) * D + CPL * qp;
+      if constexpr (CPL >= 4) {
+#pragma unroll
+        for (int j = 0; j < CPL; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
       } else {
         *reinterpret_cast<float2*>(dst) = make_float2(x[0], x[1]);
       }
