@@ -30,13 +30,16 @@
 // line, so the ldmatrix row gathers are conflict-free.
 //
 // Compact tier, per step: the same contractions in the rotated basis ("QuantForge V2
-// Walkthrough", section 1: rotate the query instead of the keys) with FP16 operands.  The
-// rotated query H q is split into an FP16 high part (S^T rows 0..7) and residual (rows
-// 8..15), so scores keep ~22 significant bits.  Code bytes become (c[lo], c[hi]) half
-// pairs through a per-lane replicated table in shared memory; V code nibbles of two
-// tokens are interleaved into one byte so one table entry is a (token, token) pair at one
-// dimension.  The key scale multiplies the scores, the value scale the weights, and the
-// merged output is rotated back with a Walsh-Hadamard transform in registers.
+// Walkthrough", section 1: rotate the query instead of the keys) with FP16 operands.
+//   S (16 tokens x 8 cols) = K_hat . Q^T   A = dequantised keys, B = the rotated query
+//   O^T (d x 8 cols)      += V_hat^T . P^T A = dequantised values, B = the weights
+// Code bytes become (c[lo], c[hi]) half pairs through a per-lane replicated table in
+// shared memory, each lookup one A-fragment entry; value code nibbles of two tokens share
+// a byte, so one entry is a (token, token) pair at one dimension.  The rotated query H q is
+// an FP16 high part and an FP16 residual (for G <= 4 head h's are columns h and h + 4, for
+// G = 8 a second product), so scores keep ~22 significant bits; the weights are split the
+// same way.  The key scale multiplies the scores, the value scale the weights, and the
+// output is rotated back with a Walsh-Hadamard transform over shuffles.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
