@@ -888,7 +888,9 @@ def main(argv=None):
     cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
     try:
         line = run_workload(args.workload, ctx, args, args.steps, args.warmup, cpu_s)
-        if args.workload == "ragged" and not args.no_per_config:
+        # the other workloads ride along on one GPU; a multi-GPU run times the headline only
+        # (every rank would otherwise pin its own 10 GB of staged history)
+        if args.workload == "ragged" and not args.no_per_config and ctx.world == 1:
             per = {}
             for name in PER_CONFIG:
                 free_device_memory()
