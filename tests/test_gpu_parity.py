@@ -260,8 +260,12 @@ def _oracle_hybrid(wl, w, b, heads=None):
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
-@pytest.mark.parametrize("T,W,d,G", [(3001, 1000, 128, 4), (1100, 300, 64, 8), (2000, 0, 128, 1)])
+@pytest.mark.parametrize("T,W,d,G", [(3001, 1000, 128, 4), (1100, 300, 64, 8), (2000, 0, 128, 1),
+                                     (1500, 200, 64, 1), (1700, 300, 128, 2), (900, 100, 64, 2),
+                                     (1200, 400, 128, 8)])
 def test_hybrid_small(akv, wlmod, cuda, variant, T, W, d, G):
+    """Every (d, G) the compact kernel is built for: its per-head lane groups hold 2 to 32
+    coordinates per lane (G = 1 at d = 64 up to G = 8 at d = 128)."""
     import torch
     wl = synth.Workload("hybrid-small", B=2, Hq=2 * G, Hkv=2, d=d, split_tokens=256, extra={"T": T, "window": W})
     w = wlmod.HybridResident(wl, cuda)
