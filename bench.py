@@ -851,13 +851,18 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
     tw1 = time.monotonic()
     sampler.stop()
     ms = ctx.max(e0.elapsed_time(e1))
+    # bytes one step's attention reads at the start of the timed steps: per KV head, K and V,
+    # a compact token is d/2 code bytes + a 2-byte norm, a window token 2d bytes
+    step_bytes = int(st.c.sum()) * wl.Hkv * 2 * (wl.d // 2 + 2) + int(st.win.sum()) * wl.Hkv * 2 * wl.d * 2
     st._state()
     aged = st.aged_blocks - aged0
     # step j attends every earlier token plus the B it appends
     tok = sum(tok0 + wl.B * (j + 1) for j in range(steps))
     value = tok * ctx.world / (ms * 1e-3)
     err = int(st.err.item())
-    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ctx.world, "steps": steps,
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (ms / steps * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ctx.world, "steps": steps,
             "warmup": warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "window aging on the hybrid shape: batch 4, 32 q / 8 KV heads, d 128, "
@@ -867,9 +872,17 @@ def run_aging(name, ctx, args, steps, warmup, cpu_s):
                        "variant": args.variant, "timing": "CUDA events around whole steps",
                        "step": "one akv_aging_step call (append, aging encode, attention launches, merge)"},
             "aged_pages_in_timed_steps": int(aged),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "kernel": "whole step (append, aging, both tiers, merge)",
+                         "algorithmic_bytes": step_bytes, "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"},
             "e2e": None, "gpu_launches": steps * 4 + 2 * int(aged > 0) * (aged // wl.B),
             # the timed steps take milliseconds: the samples within 0.25 s of them
             "clocks": sampler.summary(tw0 - 0.25, tw1 + 0.25), "device_error_word": err}
+    if ctx.rank == 0 and ctx.world == 1 and cpu_s > 0:
+        # the oracle of the hybrid shape: the aging step attends the same two tiers (its encode of
+        # one page per 16 steps is a small part of the work)
+        line["cpu_baseline"] = cpu_baseline("hybrid", base, cpu_s)
+    return line
 
 
 def run_workload(name, ctx, args, steps, warmup, cpu_s):
