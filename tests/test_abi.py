@@ -289,3 +289,24 @@ def test_aging_create_refusals(akv):
     assert refused(ring_head=[0, R]) == akv.AKV_ERR_INVALID
     assert refused(d=80) == akv.AKV_ERR_UNSUPPORTED
     assert refused(window=cmp) == akv.AKV_ERR_INVALID
+
+
+def test_paged_code_pool_keeps_a_pages_key_and_value_blocks_adjacent(akv):
+    """The paged compact pool of the ragged and aging workloads: [P][Hkv][2][block], the value
+    block of (page, head) right after its key block, strides in blocks (2 Hkv per page, 2 per
+    head); a tier over it passes the library's checks."""
+    import torch
+    from kv_cache_tiering_b200 import workloads
+    P, H, d = 5, 8, 128
+    bb = akv.codes4_block_bytes(d)
+    assert bb == 1056
+    pool, k, v, s_seq, s_head = workloads.code_page_pool(P, H, d, "cpu")
+    assert tuple(pool.shape) == (P, H, 2, bb) and (s_seq, s_head) == (2 * H, 2)
+    assert v.data_ptr() - k.data_ptr() == bb
+    # block (page p, head h) of K starts at (p * s_seq + h * s_head) blocks
+    for p, h in [(0, 0), (3, 5), (4, 7)]:
+        assert k[p, h].data_ptr() - pool.data_ptr() == (p * s_seq + h * s_head) * bb
+        assert v[p, h].data_ptr() - k[p, h].data_ptr() == bb
+    tier = akv.Tier(akv.AKV_TIER_CODES4, 0x100000, 0x100000 + bb, lens=[60], paged=True, page_table=0x200000,
+                    page_table_stride=4, n_pages=P, stride_seq=s_seq, stride_head=s_head)
+    assert akv.akv_decode_workspace_size(1, 32, H, d, [tier], 512) > 0
