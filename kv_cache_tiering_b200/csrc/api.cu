@@ -393,13 +393,14 @@ struct PlannedLaunch {
 // two kernels, alone and side by side):
 //   - a compact split runs on one warp; a 16-token step takes about 0.23 + 0.073 w us when its
 //     SM holds w busy warps (they share the SM's issue slots and shared-memory port);
-//   - a BF16 split runs on one CTA as 8 chains; a chain step takes about 1.4 us;
+//   - a BF16 split runs on one CTA as 8 chains; a chain step takes about 1.6 us;
 //   - a launch that follows another costs about 4 us of ramp and tail.
-// The share minimises the larger of the two durations (ties go to the smaller share, so the
-// BF16 tier keeps the slack).  It is used only when that beats the two launches in a row,
-// which is when one of them would leave SMs or warps idle.  Returns 0 for "in a row".
+// The share minimises the larger of the two durations; among equal estimates it is the
+// largest, so the compact tier keeps the slack.  It is used only when that beats the two
+// launches in a row, which is when one of them would leave SMs or warps idle.  Returns 0 for
+// "in a row".
 int compact_sm_share(int sms, int64_t items_c, int warps_c, int64_t steps_c, int64_t items_x, int64_t chain_steps_x) {
-  constexpr double kStepBase = 0.23, kStepPerWarp = 0.073, kBf16ChainStep = 1.4, kLaunch = 4.0;
+  constexpr double kStepBase = 0.23, kStepPerWarp = 0.073, kBf16ChainStep = 1.6, kLaunch = 4.0;
   auto t_codes = [&](int ctas) {
     const double busy = std::min<double>((double)warps_c, (double)items_c / ctas);
     return (double)ceil_div(items_c, (int64_t)warps_c * ctas) * steps_c * (kStepBase + kStepPerWarp * busy);
@@ -407,9 +408,9 @@ int compact_sm_share(int sms, int64_t items_c, int warps_c, int64_t steps_c, int
   auto t_bf16 = [&](int ctas) { return (double)ceil_div(items_x, ctas) * chain_steps_x * kBf16ChainStep; };
   int best = 0;
   double best_t = t_codes(sms) + t_bf16(sms) + kLaunch;
-  for (int share = 1; share < sms; ++share) {
+  for (int share = 1; share < sms; ++share) {  // ties go to the larger compact share
     const double t = std::max(t_codes(share), t_bf16(sms - share));
-    if (t < best_t) {
+    if (t <= best_t) {
       best_t = t;
       best = share;
     }
