@@ -96,3 +96,18 @@ def test_reference_arm_line_and_nonzero_ranks_exit_quietly():
     r1 = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"],
                     {"RANK": "1", "WORLD_SIZE": "2"})
     assert r1.returncode == 0 and r1.stdout.strip() == ""
+
+
+def test_staging_trade_arithmetic():
+    """The staged-hybrid line's trade: PCIe bytes kept off the link against GPU time added,
+    from the two staged entries of one run."""
+    bf16 = {"h2d_bytes_per_step": 8_000_000_000, "roofline": {"peak": 50.0}, "attention_gpu_ms_per_step": 7.5,
+            "ms_per_step": 160.0}
+    hyb = {"h2d_bytes_per_step": 2_000_000_000, "roofline": {"peak": 48.0}, "attention_gpu_ms_per_step": 11.0,
+           "ms_per_step": 40.0}
+    t = bench.staging_trade(bf16, hyb)
+    assert t["pcie_bytes_saved_per_step"] == 6_000_000_000
+    assert t["pcie_bytes_ratio"] == 4.0
+    assert t["pcie_ms_saved_per_step"] == pytest.approx(120.0)  # 6 GB at the BF16 run's 50 GB/s ceiling
+    assert t["gpu_ms_added_per_step"] == pytest.approx(3.5)
+    assert t["step_speedup"] == pytest.approx(4.0)
